@@ -1,0 +1,116 @@
+"""The oracle: a plain fp64 CPU statement of the Gated DeltaNet-2 recurrence.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s
+CPU-baseline leg may import this package. The CUDA library never loads it and shares no
+code with it; the two meet only through the seeded input generators.
+
+The arithmetic lives in ``gdn2_ref.c`` (one token at a time, fp64); this module only builds
+that file with gcc and marshals numpy arrays to it through ctypes. Which passage of the
+pages each step follows is stated in ``gdn2_ref.c``.
+
+Parity status: every step is pinned by ``tests/test_oracle_pins.py`` (the delta-rule post's
+worked example, closed forms, invariants and brute force); the one reading the pages leave
+open -- which side of the erase term carries b -- is pinned to the adopted form only by a
+hand-computed case.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn2_ref.c")
+_SO = os.path.join(_HERE, "libgdn2_ref.so")
+_lib = None
+
+F32, BF16 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile gdn2_ref.c into libgdn2_ref.so with gcc (OpenMP). Returns the .so path."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", _SO, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _SO
+
+
+def load():
+    """Load the oracle library. GDN2_ORACLE_LIB names another build of gdn2_ref.c to load
+    instead (the mutation test uses it to check that the pins catch planted mistakes)."""
+    global _lib
+    if _lib is None:
+        override = os.environ.get("GDN2_ORACLE_LIB")
+        if not override:
+            build()
+        lib = ctypes.CDLL(override or _SO)
+        lib.gdn2_fwd_ref.restype = ctypes.c_int
+        vp = ctypes.c_void_p
+        lib.gdn2_fwd_ref.argtypes = [ctypes.c_int, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int]
+        lib.gdn2_ref_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(load().gdn2_ref_max_threads())
+
+
+def _as_buffer(x, dtype_code):
+    """Return a C-contiguous numpy array whose raw bytes are fp32 or bf16 bit patterns."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: take its exact bits, never round
+        import torch
+        x = x.detach().cpu().contiguous()
+        if x.dtype == torch.bfloat16:
+            return np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16))
+        return np.ascontiguousarray(x.to(torch.float32).numpy())
+    x = np.asarray(x)
+    if dtype_code == BF16:
+        if x.dtype != np.uint16:
+            raise TypeError("bf16 oracle inputs must be uint16 bit patterns or torch bf16")
+        return np.ascontiguousarray(x)
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def fwd_ref(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
+            bf16=None, n_threads: int = 0, want_state: bool = True):
+    """Run the oracle. Shapes: q,k [T,Hqk,dk]; v,w [T,Hv,dv]; log_alpha,b [T,Hv,dk];
+    S0 [N,Hv,dk,dv] or None. Returns (o [T,Hv,dv] float64, S_T [N,Hv,dk,dv] float64 or None).
+
+    ``bf16`` selects the element type of q,k,v,b,w (inferred from torch tensors when None).
+    ``cu_seqlens`` [N+1] int32 packs N sequences; without it the T tokens are split into
+    ``n_seq`` equal sequences (default 1).
+    """
+    if bf16 is None:
+        bf16 = hasattr(q, "dtype") and str(q.dtype) == "torch.bfloat16"
+    code = BF16 if bf16 else F32
+    qa, ka, va, ba, wa = (_as_buffer(t, code) for t in (q, k, v, b, w))
+    la = _as_buffer(log_alpha, F32).astype(np.float32, copy=False)
+    s0 = None if S0 is None else _as_buffer(S0, F32).astype(np.float32, copy=False)
+    T, h_qk, dk = qa.shape
+    _, h_v, dv = va.shape
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int32))
+        n = cu.shape[0] - 1
+    else:
+        cu = None
+        n = 1 if n_seq is None else int(n_seq)
+    o = np.empty((T, h_v, dv), dtype=np.float64)
+    st = np.empty((n, h_v, dk, dv), dtype=np.float64) if want_state else None
+    rc = load().gdn2_fwd_ref(n, T, _ptr(cu), h_qk, h_v, dk, dv, code,
+                             _ptr(qa), _ptr(ka), _ptr(va), _ptr(la), _ptr(ba), _ptr(wa),
+                             _ptr(s0), _ptr(o), _ptr(st), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"gdn2_fwd_ref rejected its arguments (status {rc})")
+    return o, st
