@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""Benchmark of libgdn2 on B200: Gated DeltaNet-2 chunk-forward tokens/s (headline) and
+decode tokens/s, each with its HBM roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {libgdn2,reference}]
+
+A step is one gdn2_chunk_fwd over the prefill workload (batch 8, 16 heads, T=4096,
+dk=dv=128, bf16 inputs, fp32 log-decay and state). A token is one position of one sequence
+across all heads. Inputs (1.07 GB) are larger than L2, so no flush is needed between steps.
+Under torchrun every rank runs its own batch (weak scaling, no collective on the data
+path); the time is the maximum over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the oracle (fp64, CPU, OpenMP) on a bounded sample of the same
+workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "prefill_b8_h16_t4096"
+DECODE = "decode_256seq_h32"
+DECODE_TIMED_STEPS = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libgdn2", choices=["libgdn2", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.2)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.1)
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def prefill_bytes(wl, lengths) -> int:
+    """Algorithmic bytes of one chunk-forward: every input read once, o and S_T written once;
+    q and k are counted once per query/key head (value heads in a group share them)."""
+    es = torch.finfo(wl.dtype).bits // 8
+    T = int(sum(lengths))
+    per_token = (wl.h_qk * 2 * wl.dk * es
+                 + wl.h_v * (3 * wl.dv * es + wl.dk * es + 4 * wl.dk))
+    state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
+    return T * per_token + state * (2 if wl.S0_std else 1)
+
+
+def decode_bytes(wl) -> int:
+    es = torch.finfo(wl.dtype).bits // 8
+    n = wl.n_seq
+    io = n * (wl.h_qk * 2 * wl.dk * es + wl.h_v * (3 * wl.dv * es + wl.dk * es + 4 * wl.dk))
+    return io + 2 * n * wl.h_v * wl.dk * wl.dv * 4
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(seconds_target: float = 15.0):
+    """The oracle as it stands, on a bounded sample of the prefill workload: sequence 0, all
+    16 heads, the first T_s tokens (T_s grown until the run takes about seconds_target)."""
+    import oracle
+    from gated_delta_rule_160_b200 import workloads as W
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, "cpu", n_seq=1, T=wl.T)
+    threads = oracle.max_threads()
+    T_s = 64
+    while True:
+        sl = lambda x: x[:T_s].contiguous()
+        t0 = time.perf_counter()
+        oracle.fwd_ref(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["log_alpha"]), sl(d["b"]), sl(d["w"]))
+        dt = time.perf_counter() - t0
+        if dt >= seconds_target / 4 or T_s >= wl.T:
+            break
+        T_s = min(wl.T, T_s * 4)
+    return {"value": T_s / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"sequence 0 of {PREFILL}, all {wl.h_v} heads, first {T_s} tokens "
+                      f"(fp64 oracle, {dt:.1f} s)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    base = cpu_baseline(seconds_target=max(4.0, 60.0 / max(1, args.steps + args.warmup)))
+    # each step re-runs the sample; report tokens/s over the timed steps
+    import oracle
+    from gated_delta_rule_160_b200 import workloads as W
+    wl = W.WORKLOADS[PREFILL]
+    T_s = int(base["sample"].split("first ")[1].split(" ")[0])
+    d = W.prefill_inputs(wl, "cpu", n_seq=1, T=T_s)
+    run = lambda: oracle.fwd_ref(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"])
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = time.perf_counter() - t0
+    val = T_s * args.steps / dt
+    base["value"] = val
+    print(json.dumps({
+        "impl": "reference", "metric": "GDN-2 chunk-fwd tokens/s", "value": val, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL, "sample": base["sample"]},
+        "cpu_baseline": base,
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("libgdn2 needs a CUDA device")
+    import gated_delta_rule_160_b200 as G
+    from gated_delta_rule_160_b200 import workloads as W
+
+    G.load_library()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    hbm, peak_src = peaks()
+
+    # ---------------- prefill (headline)
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, dev)
+    tokens_per_step = int(sum(d["lengths"]))
+    o = torch.empty_like(d["v"])
+    S_T = torch.empty((wl.n_seq, wl.h_v, wl.dk, wl.dv), dtype=torch.float32, device=dev)
+    step = lambda: G.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=d["S0"],
+                                    n_seq=d["n_seq"], o=o, S_T=S_T, stream=stream)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_begin = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_begin.record(stream)
+        for i in range(args.steps):
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_local = t_begin.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    kern_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    value = world * tokens_per_step / (ms / 1000.0)
+    nbytes = prefill_bytes(wl, d["lengths"])
+    achieved = nbytes / (kern_ms / 1000.0) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": None,
+                "peak_source": f"{peak_src} hbm_gbs", "kernel": "gdn2 chunk-forward",
+                "algorithmic_bytes_per_launch": nbytes}
+
+    # ---------------- decode (the second metric)
+    dwl = W.WORKLOADS[DECODE]
+    S = W.decode_state(dwl, dev)
+    dec_in = [W.decode_inputs(dwl, s, dev) for s in range(4)]
+    do = torch.empty_like(dec_in[0]["v"])
+    dstep = lambda i: G.gdn2_decode_step(*(dec_in[i % 4][k] for k in ("q", "k", "v", "log_alpha", "b", "w")),
+                                         S, o=do, stream=stream)
+    for i in range(5):
+        dstep(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(DECODE_TIMED_STEPS):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dms = max_over_ranks(e0.elapsed_time(e1) / DECODE_TIMED_STEPS, world)
+    dbytes = decode_bytes(dwl)
+    dach = dbytes / (dms / 1000.0) / 1e9
+    decode = {"metric": "GDN-2 decode tokens/s", "value": world * dwl.n_seq / (dms / 1000.0),
+              "unit": "tokens/s", "ms_per_step": dms, "steps": DECODE_TIMED_STEPS,
+              "config": {"workload": DECODE, "n_seq": dwl.n_seq, "heads": dwl.h_v, "dk": dwl.dk,
+                         "dv": dwl.dv, "state_bytes": dwl.n_seq * dwl.h_v * dwl.dk * dwl.dv * 4},
+              "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
+                           "frac": dach / hbm, "traffic": None,
+                           "peak_source": f"{peak_src} hbm_gbs",
+                           "algorithmic_bytes_per_launch": dbytes}}
+    del S, dec_in
+
+    # ---------------- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        names = ("q", "k", "v", "log_alpha", "b", "w")
+        host = {k: d[k].cpu().pin_memory() for k in names}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_host.numel() * o_host.element_size()
+        dev_in = {k: torch.empty_like(d[k]) for k in names}
+        del d
+
+        def e2e_step():
+            for k in names:
+                dev_in[k].copy_(host[k], non_blocking=True)
+            G.gdn2_chunk_fwd(*(dev_in[k] for k in names), n_seq=wl.n_seq, o=o, S_T=S_T, stream=stream)
+            o_host.copy_(o, non_blocking=True)
+            stream.synchronize()
+
+        for _ in range(2):
+            e2e_step()
+        n_e2e = max(3, min(args.steps, 10))
+        barrier(world)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(a.elapsed_time(b_) / n_e2e, world)
+        e2e = {"value": world * tokens_per_step / (ems / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems,
+               "steps": n_e2e}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": "GDN-2 chunk-fwd tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": PREFILL, "global_batch": wl.n_seq * world, "seq_len": wl.T,
+                       "heads": wl.h_v, "dk": wl.dk, "dv": wl.dv, "parallelism": f"replicas{world}",
+                       "inputs": "bf16 q,k,v,b,w; fp32 log_alpha and state",
+                       "l2": "inputs (1.07 GB per rank) larger than L2; no flush"},
+            "roofline": roofline,
+            "decode": decode,
+            "e2e": e2e,
+            "cpu_baseline": base,
+            "clocks": clocks.summary(),
+            "gpu_launches": args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

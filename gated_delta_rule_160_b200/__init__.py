@@ -1,0 +1,133 @@
+"""libgdn2: the Gated DeltaNet-2 state recurrence on B200 (sm_100a).
+
+This package is a thin ctypes binding over the C ABI declared in ``include/gdn2.h``; every
+step of the recurrence runs in the CUDA kernels of ``libgdn2.so``. PyTorch provides device
+memory and streams only. There is no CPU fallback: if the library is missing or fails to
+load, importing the functions below raises.
+
+    gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, ...) -> (o, S_T)
+    gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None) -> o     (S updated in place)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgdn2.so")
+
+GDN2_F32, GDN2_BF16 = 0, 1
+STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_CUDA"}
+ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_decode_step",
+                 "gdn2_last_error_string", "gdn2_version")
+
+
+class Gdn2Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("n_seq", ctypes.c_int), ("T_total", ctypes.c_int), ("h_qk", ctypes.c_int),
+                ("h_v", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
+                ("dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libgdn2.so (built by ``python -m gated_delta_rule_160_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m gated_delta_rule_160_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz = ctypes.c_void_p, ctypes.c_size_t
+    lib.gdn2_chunk_fwd_workspace_size.restype = sz
+    lib.gdn2_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
+    lib.gdn2_chunk_fwd.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd.argtypes = [ctypes.POINTER(Shape)] + [vp] * 10 + [vp, sz, vp]
+    lib.gdn2_decode_step.restype = ctypes.c_int
+    lib.gdn2_decode_step.argtypes = [ctypes.POINTER(Shape)] + [vp] * 9
+    lib.gdn2_last_error_string.restype = ctypes.c_char_p
+    lib.gdn2_last_error_string.argtypes = []
+    lib.gdn2_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int):
+    if status != 0:
+        msg = load_library().gdn2_last_error_string().decode()
+        raise Gdn2Error(status, msg)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GDN2_BF16
+    if t.dtype == torch.float32:
+        return GDN2_F32
+    raise TypeError(f"unsupported element type {t.dtype}; use bfloat16 or float32")
+
+
+def make_shape(q, v, n_seq: int) -> Shape:
+    T, h_qk, dk = q.shape
+    _, h_v, dv = v.shape
+    return Shape(int(n_seq), int(T), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v))
+
+
+def gdn2_chunk_fwd_workspace_size(shape: Shape, varlen: bool) -> int:
+    return int(load_library().gdn2_chunk_fwd_workspace_size(ctypes.byref(shape), int(bool(varlen))))
+
+
+def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
+                   o=None, S_T=None, want_state: bool = True, workspace=None, stream=None):
+    """Prefill: run the recurrence over whole (packed) sequences on the GPU.
+
+    q,k [T,Hqk,dk]; v,w [T,Hv,dv]; log_alpha (fp32), b [T,Hv,dk]; S0 fp32 [N,Hv,dk,dv] or
+    None; cu_seqlens int32 [N+1] or None (then ``n_seq`` equal sequences, default 1).
+    Returns (o [T,Hv,dv] in v's dtype, S_T fp32 [N,Hv,dk,dv] or None). Tensors must be
+    contiguous CUDA tensors; nothing is converted or copied here.
+    """
+    lib = load_library()
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
+    shape = make_shape(q, v, n)
+    T, h_v, dv = v.shape
+    if o is None:
+        o = torch.empty((T, h_v, dv), dtype=v.dtype, device=v.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((n, h_v, q.shape[2], dv), dtype=torch.float32, device=v.device)
+    need = gdn2_chunk_fwd_workspace_size(shape, cu_seqlens is not None)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.gdn2_chunk_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                              _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
+                              _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    return o, S_T
+
+
+def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None):
+    """One decode token per sequence: q,k [N,Hqk,dk]; v,w [N,Hv,dv]; log_alpha, b [N,Hv,dk];
+    S fp32 [N,Hv,dk,dv] updated in place. Returns o [N,Hv,dv]."""
+    lib = load_library()
+    shape = make_shape(q, v, q.shape[0])
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    _check(lib.gdn2_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream_handle(stream)))
+    return o

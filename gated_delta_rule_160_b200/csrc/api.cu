@@ -1,0 +1,170 @@
+// api.cu -- the C ABI of libgdn2 (include/gdn2.h): argument checks and kernel dispatch.
+//
+// Every check runs on the host before anything is queued; a rejected call queues
+// nothing. Error text is kept per calling thread.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "internal.cuh"
+
+namespace gdn2 {
+namespace {
+
+thread_local char g_err[512] = "";
+
+gdn2_status fail(gdn2_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+gdn2_status ok() {
+    g_err[0] = '\0';
+    return GDN2_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+// A pointer the GPU can dereference as device memory (plain or managed allocations).
+bool is_device_ptr(const void* ptr) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error this query may leave
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+gdn2_status check_shape(const gdn2_shape* sh) {
+    if (!sh) return fail(GDN2_ERR_INVALID_ARG, "shape is NULL");
+    if (sh->n_seq < 1 || sh->n_seq > 65535)
+        return fail(GDN2_ERR_INVALID_ARG, "n_seq = %d outside [1, 65535]", sh->n_seq);
+    if (sh->T_total < 0) return fail(GDN2_ERR_INVALID_ARG, "T_total = %d is negative", sh->T_total);
+    if (sh->h_qk < 1 || sh->h_v < 1)
+        return fail(GDN2_ERR_INVALID_ARG, "head counts must be positive (h_qk=%d, h_v=%d)", sh->h_qk, sh->h_v);
+    if (sh->h_v % sh->h_qk != 0)
+        return fail(GDN2_ERR_INVALID_ARG, "h_v = %d is not a multiple of h_qk = %d", sh->h_v, sh->h_qk);
+    if (sh->h_v > 65535) return fail(GDN2_ERR_UNSUPPORTED, "h_v = %d above 65535", sh->h_v);
+    if (sh->dtype != GDN2_F32 && sh->dtype != GDN2_BF16)
+        return fail(GDN2_ERR_INVALID_ARG, "unknown dtype %d", (int)sh->dtype);
+    if ((sh->dk != 64 && sh->dk != 128) || (sh->dv != 64 && sh->dv != 128))
+        return fail(GDN2_ERR_UNSUPPORTED, "dk = %d, dv = %d: only 64 and 128 are supported", sh->dk, sh->dv);
+    return GDN2_OK;
+}
+
+struct NamedPtr {
+    const char* name;
+    const void* ptr;
+    bool required;
+};
+
+gdn2_status check_ptrs(const NamedPtr* ps, int n) {
+    for (int i = 0; i < n; ++i) {
+        if (!ps[i].ptr) {
+            if (ps[i].required) return fail(GDN2_ERR_INVALID_ARG, "%s is NULL", ps[i].name);
+            continue;
+        }
+        if (!aligned16(ps[i].ptr))
+            return fail(GDN2_ERR_INVALID_ARG, "%s = %p is not 16-byte aligned", ps[i].name, ps[i].ptr);
+        if (!is_device_ptr(ps[i].ptr))
+            return fail(GDN2_ERR_INVALID_ARG, "%s = %p is not device memory", ps[i].name, ps[i].ptr);
+    }
+    return GDN2_OK;
+}
+
+Params make_params(const gdn2_shape* sh, const void* q, const void* k, const void* v,
+                   const float* la, const void* b, const void* w, const float* S0,
+                   const int32_t* cu, void* o, float* S_T) {
+    Params p{};
+    p.n_seq = sh->n_seq;
+    p.T_total = sh->T_total;
+    p.h_qk = sh->h_qk;
+    p.h_v = sh->h_v;
+    p.dk = sh->dk;
+    p.dv = sh->dv;
+    p.T_fixed = cu ? 0 : sh->T_total / sh->n_seq;
+    p.q = q; p.k = k; p.v = v; p.log_alpha = la; p.b = b; p.w = w;
+    p.S0 = S0; p.cu_seqlens = cu; p.o = o; p.S_T = S_T; p.order = nullptr;
+    return p;
+}
+
+}  // namespace
+}  // namespace gdn2
+
+using namespace gdn2;
+
+extern "C" {
+
+const char* gdn2_last_error_string(void) { return g_err; }
+
+int gdn2_version(void) { return 100; }
+
+size_t gdn2_chunk_fwd_workspace_size(const gdn2_shape* shape, int varlen) {
+    if (!shape || !varlen || shape->n_seq < 1) return 0;
+    // the longest-first order of the sequences, 256-byte rounded
+    return ((size_t)shape->n_seq * sizeof(int32_t) + 255) & ~(size_t)255;
+}
+
+gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const void* b, const void* w, const float* S0,
+                           const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
+                           size_t workspace_bytes, gdn2_stream_t stream) {
+    gdn2_status st = check_shape(shape);
+    if (st != GDN2_OK) return st;
+    const bool any_tokens = shape->T_total > 0;
+    const NamedPtr ps[] = {
+        {"q", q, any_tokens}, {"k", k, any_tokens}, {"v", v, any_tokens},
+        {"log_alpha", log_alpha, any_tokens}, {"b", b, any_tokens}, {"w", w, any_tokens},
+        {"o", o, any_tokens}, {"S0", S0, false}, {"S_T", S_T, false},
+        {"cu_seqlens", cu_seqlens, false}, {"workspace", workspace, false},
+    };
+    st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
+    if (st != GDN2_OK) return st;
+    if (!cu_seqlens && shape->T_total % shape->n_seq != 0)
+        return fail(GDN2_ERR_INVALID_ARG, "T_total = %d is not a multiple of n_seq = %d (and no cu_seqlens)",
+                    shape->T_total, shape->n_seq);
+    const size_t need = gdn2_chunk_fwd_workspace_size(shape, cu_seqlens != nullptr);
+    if (need && (!workspace || workspace_bytes < need))
+        return fail(GDN2_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(GDN2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+
+    Params p = make_params(shape, q, k, v, log_alpha, b, w, S0, cu_seqlens, o, S_T);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cu_seqlens) {
+        int32_t* order = static_cast<int32_t*>(workspace);
+        cudaError_t e = launch_varlen_order(p, order, s);
+        if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "order kernel: %s", cudaGetErrorString(e));
+        p.order = order;
+    }
+    cudaError_t e = launch_recurrent(p, shape->dtype, s);
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+gdn2_status gdn2_decode_step(const gdn2_shape* shape, const void* q, const void* k, const void* v,
+                             const float* log_alpha, const void* b, const void* w, float* S, void* o,
+                             gdn2_stream_t stream) {
+    gdn2_status st = check_shape(shape);
+    if (st != GDN2_OK) return st;
+    if (shape->T_total != shape->n_seq)
+        return fail(GDN2_ERR_INVALID_ARG, "decode takes one token per sequence: T_total = %d, n_seq = %d",
+                    shape->T_total, shape->n_seq);
+    if ((long long)shape->n_seq * shape->h_v > 0x7fffffffLL)
+        return fail(GDN2_ERR_UNSUPPORTED, "n_seq * h_v too large for one launch");
+    const NamedPtr ps[] = {
+        {"q", q, true}, {"k", k, true}, {"v", v, true}, {"log_alpha", log_alpha, true},
+        {"b", b, true}, {"w", w, true}, {"S", S, true}, {"o", o, true},
+    };
+    st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
+    if (st != GDN2_OK) return st;
+    Params p = make_params(shape, q, k, v, log_alpha, b, w, nullptr, nullptr, o, S);
+    cudaError_t e = launch_decode(p, shape->dtype, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// internal.cuh -- declarations shared by the libgdn2 translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn2.h"
+
+namespace gdn2 {
+
+// Everything a kernel needs about one call; pointers are device pointers.
+struct Params {
+    int n_seq, T_total, h_qk, h_v, dk, dv;
+    int T_fixed;               // tokens per sequence when cu_seqlens is NULL, else 0
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const void* b;
+    const void* w;
+    const float* S0;           // nullable
+    const int32_t* cu_seqlens; // nullable
+    void* o;
+    float* S_T;                // nullable (decode: the in/out state)
+    const int32_t* order;      // nullable: sequences longest first (varlen scheduling)
+};
+
+// Token range [t0, t1) of sequence n.
+__device__ __forceinline__ void seq_bounds(const Params& p, int n, int& t0, int& t1) {
+    if (p.cu_seqlens) {
+        // clamped, so malformed offsets cannot send a kernel outside the token range
+        t0 = min(max(p.cu_seqlens[n], 0), p.T_total);
+        t1 = min(max(p.cu_seqlens[n + 1], t0), p.T_total);
+    } else {
+        t0 = n * p.T_fixed;
+        t1 = t0 + p.T_fixed;
+    }
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, cudaStream_t s);
+cudaError_t launch_decode(const Params& p, gdn2_dtype dt, cudaStream_t s);
+cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s);
+
+}  // namespace gdn2

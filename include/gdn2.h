@@ -1,0 +1,125 @@
+/*
+ * gdn2.h -- C ABI of libgdn2, the sm_100a (B200) implementation of the Gated DeltaNet-2
+ * state recurrence.
+ *
+ * The operation (per sequence n and value head h; tokens t in order):
+ *   S'_t = Diag(alpha_t) S_{t-1},  alpha_t = exp(log_alpha_t)     channel-wise decay, key axis
+ *   r_t  = S'_t^T k_t                                              key read of the old state
+ *   S_t  = S'_t - (b_t (.) k_t) r_t^T + k_t (w_t (.) v_t)^T        erase (key axis), write (value axis)
+ *   o_t  = S_t^T q_t                                               query read of the updated state
+ * Sources: the tilnote.io note on Gated DeltaNet-2, section "Gated DeltaNet-2 design
+ * point" (a channel-wise erase gate b_t on the key axis, a channel-wise write gate w_t on
+ * the value axis, the KDA channel-wise decay; decay, then remove the key-side component,
+ * then add the value-side component); the ai-systems-engineering.com post "Delta rule:
+ * correcting the state's associations toward the new Value", sections "Why read with the
+ * Key, why with the Query" and "Recording the difference between the read value and the
+ * new Value" (key read before the edit, query read after it, r^T = k^T S, rows of S are
+ * key channels and columns value channels); the Gated DeltaNet wiki page
+ * (aiki.softdaddy-o.com), section "How it works" (query/key heads shared by groups of
+ * value heads). No scale is applied to q.
+ *
+ * Layouts (row-major, innermost index last, every tensor contiguous):
+ *   q, k        [T_total, h_qk, dk]   dtype
+ *   v, w, o     [T_total, h_v,  dv]   dtype (o is written in the dtype of v)
+ *   log_alpha   [T_total, h_v,  dk]   float32
+ *   b           [T_total, h_v,  dk]   dtype
+ *   S0, S_T, S  [n_seq, h_v, dk, dv]  float32 (dv contiguous)
+ *   cu_seqlens  [n_seq + 1] int32     packed sequence offsets (0, ..., T_total)
+ * dtype GDN2_BF16 means bfloat16; GDN2_F32 means float32 for q, k, v, b, w and o.
+ * Value head h reads query/key head h / (h_v / h_qk).
+ *
+ * Ownership: every tensor pointer is a device pointer owned by the caller and must stay
+ * valid until the work queued on `stream` has finished. The library allocates no device
+ * memory. Calls are asynchronous on `stream` (0 = the legacy default stream); nothing is
+ * synchronised.
+ *
+ * Errors: arguments are checked on the host before anything is queued. A rejected call
+ * queues nothing and returns GDN2_ERR_INVALID_ARG (bad pointer, size, alignment,
+ * layout) or GDN2_ERR_UNSUPPORTED (a valid shape these kernels do not handle); a
+ * failed launch returns GDN2_ERR_CUDA. gdn2_last_error_string() describes the last
+ * failure of the calling thread. Nothing is thrown or aborted across the ABI.
+ *
+ * Supported: dk, dv in {64, 128}; h_v a multiple of h_qk; every pointer 16-byte aligned.
+ */
+#ifndef GDN2_H
+#define GDN2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GDN2_API __attribute__((visibility("default")))
+#else
+#define GDN2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gdn2_stream_t; /* a cudaStream_t */
+
+typedef enum { GDN2_F32 = 0, GDN2_BF16 = 1 } gdn2_dtype;
+
+typedef enum {
+    GDN2_OK = 0,
+    GDN2_ERR_INVALID_ARG = 1,
+    GDN2_ERR_UNSUPPORTED = 2,
+    GDN2_ERR_CUDA = 3
+} gdn2_status;
+
+typedef struct {
+    int n_seq;        /* sequences in the batch (>= 1) */
+    int T_total;      /* packed tokens over all sequences (>= 0) */
+    int h_qk;         /* query/key heads */
+    int h_v;          /* value heads (a multiple of h_qk) */
+    int dk;           /* key channels per head: 64 or 128 */
+    int dv;           /* value channels per head: 64 or 128 */
+    gdn2_dtype dtype; /* element type of q, k, v, b, w, o */
+} gdn2_shape;
+
+/*
+ * Bytes of device workspace gdn2_chunk_fwd needs for this shape and cu_seqlens choice
+ * (varlen = 1 when a cu_seqlens pointer will be passed). 0 means no workspace.
+ */
+GDN2_API size_t gdn2_chunk_fwd_workspace_size(const gdn2_shape* shape, int varlen);
+
+/*
+ * Prefill over whole sequences (chunkwise-parallel; the recurrence above for every
+ * token). Sequences are packed by cu_seqlens; with cu_seqlens == NULL, T_total must be a
+ * multiple of n_seq and sequence n is tokens [n*T, (n+1)*T), T = T_total / n_seq.
+ * S0 == NULL starts every sequence from a zero state. S_T == NULL skips the final state.
+ * A zero-length sequence writes S_T = S0 (or 0) and no output.
+ * workspace: device memory of at least gdn2_chunk_fwd_workspace_size() bytes, 256-byte
+ * aligned, owned by the caller, reused freely after the call's work completes; may be
+ * NULL when that size is 0.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape,
+                           const void* q, const void* k, const void* v,
+                           const float* log_alpha, const void* b, const void* w,
+                           const float* S0, const int32_t* cu_seqlens,
+                           void* o, float* S_T,
+                           void* workspace, size_t workspace_bytes,
+                           gdn2_stream_t stream);
+
+/*
+ * One decode step: one new token for each of the n_seq sequences (shape->T_total must
+ * equal shape->n_seq; token n belongs to sequence n). The state S [n_seq, h_v, dk, dv] is
+ * read and updated in place; o receives the query read of the updated state.
+ */
+GDN2_API gdn2_status gdn2_decode_step(const gdn2_shape* shape,
+                             const void* q, const void* k, const void* v,
+                             const float* log_alpha, const void* b, const void* w,
+                             float* S, void* o, gdn2_stream_t stream);
+
+/* Description of the calling thread's last failure ("" if none). Never NULL. */
+GDN2_API const char* gdn2_last_error_string(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+GDN2_API int gdn2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN2_H */

@@ -1,0 +1,86 @@
+"""Host-side checks of the C ABI (no GPU needed): both libraries load, every function the
+headers in include/ declare is exported, and argument checks that run before any device
+work reject bad calls with the documented status."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn2_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_160_b200 import build
+    build.build()
+    import gated_delta_rule_160_b200 as g
+    return g.load_library()
+
+
+def test_product_library_exports_every_declared_function(lib):
+    names = _declared("gdn2.h")
+    assert {"gdn2_chunk_fwd", "gdn2_decode_step", "gdn2_chunk_fwd_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"libgdn2.so does not export {n}"
+
+
+def test_oracle_library_exports_every_declared_function(oracle_mod):
+    lib = oracle_mod.load()
+    for n in _declared("gdn2_ref.h"):
+        assert hasattr(lib, n), f"libgdn2_ref.so does not export {n}"
+
+
+def test_libraries_share_no_symbols(lib, oracle_mod):
+    """The oracle and the CUDA library are separate: neither exports the other's entry points."""
+    assert not hasattr(lib, "gdn2_fwd_ref")
+    assert not hasattr(oracle_mod.load(), "gdn2_chunk_fwd")
+
+
+def _shape(g, **kw):
+    d = dict(n_seq=1, T_total=64, h_qk=1, h_v=1, dk=64, dv=64, dtype=g.GDN2_BF16)
+    d.update(kw)
+    return g.Shape(**d)
+
+
+def _call_chunk(g, lib, shape, ptr=None):
+    p = ctypes.c_void_p(ptr) if ptr else None
+    return lib.gdn2_chunk_fwd(ctypes.byref(shape) if shape is not None else None,
+                              p, p, p, p, p, p, None, None, p, None, None, 0, None)
+
+
+def test_rejects_before_device_work(lib):
+    import gated_delta_rule_160_b200 as g
+    assert lib.gdn2_chunk_fwd(None, *([None] * 10), None, 0, None) == 1
+    assert b"shape is NULL" in lib.gdn2_last_error_string()
+    assert _call_chunk(g, lib, _shape(g, dk=96)) == 2
+    assert b"dk = 96" in lib.gdn2_last_error_string()
+    assert _call_chunk(g, lib, _shape(g, h_qk=3, h_v=4)) == 1
+    assert _call_chunk(g, lib, _shape(g, n_seq=0)) == 1
+    assert _call_chunk(g, lib, _shape(g, dtype=7)) == 1
+    assert _call_chunk(g, lib, _shape(g)) == 1  # NULL tensors with T_total > 0
+    assert b"q is NULL" in lib.gdn2_last_error_string()
+    assert _call_chunk(g, lib, _shape(g), ptr=0x1008) == 1  # misaligned
+    assert b"16-byte aligned" in lib.gdn2_last_error_string()
+    # decode: exactly one token per sequence
+    sh = _shape(g, n_seq=4, T_total=5)
+    assert lib.gdn2_decode_step(ctypes.byref(sh), *([None] * 9)) == 1
+    assert b"one token per sequence" in lib.gdn2_last_error_string()
+
+
+def test_workspace_size(lib):
+    import gated_delta_rule_160_b200 as g
+    sh = _shape(g, n_seq=64)
+    assert lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(sh), 0) == 0
+    ws = lib.gdn2_chunk_fwd_workspace_size(ctypes.byref(sh), 1)
+    assert ws >= 64 * 4 and ws % 256 == 0
+
+
+def test_version(lib):
+    assert lib.gdn2_version() >= 100

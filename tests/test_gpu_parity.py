@@ -1,0 +1,191 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, element by element.
+
+Small cases run the whole tensor through the oracle; full-size workloads are run on the
+GPU in the configuration the benchmark times and compared on sampled (sequence, head)
+pairs that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_160_b200 import workloads as W
+from tests.parity import TOL, oracle_on, rel_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    import gated_delta_rule_160_b200 as g
+    g.load_library()
+    assert torch.cuda.is_available()
+    return g
+
+
+def _compare(g, oracle_mod, d, dtype, seqs=None, qk_heads=None, label=""):
+    o, st = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=d["S0"],
+                             cu_seqlens=d["cu_seqlens"], n_seq=d["n_seq"])
+    torch.cuda.synchronize()
+    ref = oracle_on(oracle_mod, d, seqs=seqs, qk_heads=qk_heads)
+    starts = np.concatenate([[0], np.cumsum(d["lengths"])])
+    o_got = [o[starts[n]:starts[n + 1], h] for (n, h) in ref]
+    o_ref = [ref[key][0] for key in ref]
+    s_got = [st[n, h] for (n, h) in ref]
+    s_ref = [ref[key][1] for key in ref]
+    eo = rel_err(torch.cat([x.float() for x in o_got]) if o_got else torch.zeros(0),
+                 np.concatenate(o_ref) if o_ref else np.zeros(0))
+    es = rel_err(torch.stack(s_got), np.stack(s_ref))
+    tol = TOL[dtype]
+    print(f"{label}: o err {eo:.3e}, S_T err {es:.3e} (tol {tol})")
+    assert eo <= tol, f"{label}: output error {eo:.3e} > {tol}"
+    assert es <= tol, f"{label}: state error {es:.3e} > {tol}"
+    return o, st
+
+
+def test_tiny_fp32_full(g, oracle_mod):
+    wl = W.WORKLOADS["tiny_fp32"]
+    d = W.prefill_inputs(wl, "cuda")
+    _compare(g, oracle_mod, d, torch.float32, label="tiny_fp32")
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 300])
+def test_small_bf16_fixed(g, oracle_mod, T):
+    wl = W.WORKLOADS["prefill_b8_h16_t4096"]
+    d = W.prefill_inputs(wl, "cuda", n_seq=2, T=T)
+    # keep two heads of each tensor to stay small; slicing keeps the recipe's values
+    for key in ("q", "k", "v", "log_alpha", "b", "w"):
+        d[key] = d[key][:, :2].contiguous()
+    _compare(g, oracle_mod, d, torch.bfloat16, label=f"bf16 T={T}")
+
+
+def test_small_grouped_with_state(g, oracle_mod):
+    wl = W.WORKLOADS["grouped_b2_qk16_v32_t32768"]
+    d = W.prefill_inputs(wl, "cuda", T=200)
+    for key in ("q", "k"):
+        d[key] = d[key][:, :2].contiguous()
+    for key in ("v", "log_alpha", "b", "w"):
+        d[key] = d[key][:, :4].contiguous()
+    d["S0"] = d["S0"][:, :4].contiguous()
+    _compare(g, oracle_mod, d, torch.bfloat16, label="grouped small")
+
+
+def test_small_varlen_with_edges(g, oracle_mod):
+    lens = [0, 1, 63, 64, 65, 200, 0, 130]
+    T = sum(lens)
+    d = W.token_inputs(T, 2, 2, 128, 128, torch.bfloat16, "cuda", seed=77)
+    d["S0"] = W.state_input(len(lens), 2, 128, 128, 0.05, "cuda", seed=77)
+    d["cu_seqlens"] = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    d["n_seq"] = None
+    d["lengths"] = lens
+    _, st = _compare(g, oracle_mod, d, torch.bfloat16, label="varlen small")
+    # zero-length sequences return their initial state exactly
+    torch.testing.assert_close(st[0], d["S0"][0], rtol=0, atol=0)
+    torch.testing.assert_close(st[6], d["S0"][6], rtol=0, atol=0)
+
+
+def test_fp32_dk64_dv128_and_no_state_outputs(g, oracle_mod):
+    d = W.token_inputs(150, 1, 2, 64, 128, torch.float32, "cuda", seed=5)
+    d.update(S0=None, cu_seqlens=None, n_seq=1, lengths=[150])
+    _compare(g, oracle_mod, d, torch.float32, label="fp32 dk64 dv128")
+    o, st = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], want_state=False)
+    assert st is None and o.shape == d["v"].shape
+
+
+def test_empty_input(g):
+    d = W.token_inputs(0, 2, 2, 64, 64, torch.bfloat16, "cuda", seed=1)
+    S0 = W.state_input(3, 2, 64, 64, 0.1, "cuda", seed=1)
+    cu = torch.zeros(4, dtype=torch.int32, device="cuda")
+    o, st = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=S0, cu_seqlens=cu)
+    torch.cuda.synchronize()
+    assert o.numel() == 0
+    torch.testing.assert_close(st, S0, rtol=0, atol=0)
+
+
+def test_rejects_host_memory(g):
+    d = W.token_inputs(64, 1, 1, 64, 64, torch.bfloat16, "cpu", seed=1)
+    with pytest.raises(g.Gdn2Error, match="not device memory"):
+        g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"],
+                         o=torch.empty(64, 1, 64, dtype=torch.bfloat16, device="cuda"), want_state=False)
+
+
+# ------------------------------------------------------------------ decode
+
+def _decode_vs_oracle(g, oracle_mod, wl, n_seq, steps, heads=None, sample=None):
+    S = W.decode_state(wl, "cuda", n_seq=n_seq)
+    if heads is not None:
+        S = S[:, :heads].contiguous()
+    S_init = S.clone()
+    H = S.shape[1]
+    pairs = sample or [(n, h) for n in range(n_seq) for h in range(H)]
+    idx_n = torch.tensor([p[0] for p in pairs], device="cuda")
+    idx_h = torch.tensor([p[1] for p in pairs], device="cuda")
+    hist = {key: [] for key in ("q", "k", "v", "log_alpha", "b", "w", "o")}
+    for step in range(steps):
+        d = W.decode_inputs(wl, step, "cuda", n_seq=n_seq)
+        if heads is not None:
+            for key in d:
+                d[key] = d[key][:, :heads].contiguous()
+        o = g.gdn2_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S)
+        d["o"] = o
+        for key in hist:  # keep only the sampled (sequence, head) slices
+            hist[key].append(d[key][idx_n, idx_h].cpu())
+    torch.cuda.synchronize()
+    got_o, ref_o, got_s, ref_s = [], [], [], []
+    for i, (n, h) in enumerate(pairs):
+        # the decode steps of sequence n are one sequence of `steps` tokens for the oracle
+        seq = {key: torch.stack([x[i] for x in hist[key]])[:, None] for key in hist}
+        o_ref, s_ref = oracle_mod.fwd_ref(seq["q"], seq["k"], seq["v"], seq["log_alpha"], seq["b"],
+                                          seq["w"], S0=S_init[n:n + 1, h:h + 1].cpu())
+        got_o.append(seq["o"][:, 0].float())
+        ref_o.append(o_ref[:, 0])
+        got_s.append(S[n, h].cpu())
+        ref_s.append(s_ref[0, 0])
+    eo = rel_err(torch.stack(got_o), np.stack(ref_o))
+    es = rel_err(torch.stack(got_s), np.stack(ref_s))
+    print(f"decode {n_seq}x{steps}: o err {eo:.3e}, S err {es:.3e}")
+    tol = TOL[wl.dtype]
+    assert eo <= tol and es <= tol
+
+
+def test_decode_small(g, oracle_mod):
+    wl = W.WORKLOADS["decode_256seq_h32"]
+    _decode_vs_oracle(g, oracle_mod, wl, n_seq=4, steps=20, heads=3)
+
+
+def test_decode_equals_chunk_fwd(g):
+    """T decode steps from S0 equal one prefill over the same T tokens from S0."""
+    T, H, dk, dv = 40, 2, 128, 128
+    d = W.token_inputs(T, H, H, dk, dv, torch.float32, "cuda", seed=3)
+    S0 = W.state_input(1, H, dk, dv, 0.05, "cuda", seed=3)
+    o_ref, s_ref = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=S0)
+    S = S0.clone()
+    outs = []
+    for t in range(T):
+        outs.append(g.gdn2_decode_step(*(d[key][t:t + 1] for key in ("q", "k", "v", "log_alpha", "b", "w")), S))
+    torch.cuda.synchronize()
+    torch.testing.assert_close(torch.cat(outs), o_ref, rtol=1e-4, atol=1e-5)
+    torch.testing.assert_close(S, s_ref, rtol=1e-4, atol=1e-5)
+
+
+# ------------------------------------------------------------------ full-size, sampled
+
+@pytest.mark.parametrize("name,seqs,qk_heads", [
+    ("prefill_b8_h16_t4096", [0, 7], [0, 15]),
+    ("grouped_b2_qk16_v32_t32768", [1], [5]),
+    ("varlen_64seq_h16", None, [3]),   # None: the longest and the shortest sequence
+])
+def test_full_size_sampled(g, oracle_mod, name, seqs, qk_heads):
+    wl = W.WORKLOADS[name]
+    d = W.prefill_inputs(wl, "cuda")
+    if seqs is None:
+        lens = d["lengths"]
+        seqs = [int(np.argmax(lens)), int(np.argmin(lens))]
+    _compare(g, oracle_mod, d, wl.dtype, seqs=seqs, qk_heads=qk_heads, label=name)
+
+
+def test_decode_full_size_sampled(g, oracle_mod):
+    """All 256 x 32 states through all 512 steps on the GPU; the oracle replays sampled
+    (sequence, head) pairs as 512-token sequences."""
+    wl = W.WORKLOADS["decode_256seq_h32"]
+    _decode_vs_oracle(g, oracle_mod, wl, n_seq=wl.n_seq, steps=wl.decode_steps,
+                      sample=[(0, 0), (255, 31), (100, 17)])
