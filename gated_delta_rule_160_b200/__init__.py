@@ -33,7 +33,7 @@ class Gdn2Error(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("n_seq", ctypes.c_int), ("T_total", ctypes.c_int), ("h_qk", ctypes.c_int),
                 ("h_v", ctypes.c_int), ("dk", ctypes.c_int), ("dv", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("o_dtype", ctypes.c_int)]
 
 
 _lib = None
@@ -76,18 +76,19 @@ def _check(status: int):
         raise Gdn2Error(status, msg)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
-    if t.dtype == torch.bfloat16:
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
         return GDN2_BF16
-    if t.dtype == torch.float32:
+    if dt == torch.float32:
         return GDN2_F32
-    raise TypeError(f"unsupported element type {t.dtype}; use bfloat16 or float32")
+    raise TypeError(f"unsupported element type {dt}; use bfloat16 or float32")
 
 
-def make_shape(q, v, n_seq: int) -> Shape:
+def make_shape(q, v, n_seq: int, out_dtype=torch.float32) -> Shape:
     T, h_qk, dk = q.shape
     _, h_v, dv = v.shape
-    return Shape(int(n_seq), int(T), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v))
+    return Shape(int(n_seq), int(T), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v.dtype),
+                 _dtype_code(out_dtype))
 
 
 def gdn2_chunk_fwd_workspace_size(shape: Shape, varlen: bool) -> int:
@@ -95,20 +96,23 @@ def gdn2_chunk_fwd_workspace_size(shape: Shape, varlen: bool) -> int:
 
 
 def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
-                   o=None, S_T=None, want_state: bool = True, workspace=None, stream=None):
+                   o=None, S_T=None, want_state: bool = True, workspace=None, stream=None,
+                   out_dtype=torch.float32):
     """Prefill: run the recurrence over whole (packed) sequences on the GPU.
 
     q,k [T,Hqk,dk]; v,w [T,Hv,dv]; log_alpha (fp32), b [T,Hv,dk]; S0 fp32 [N,Hv,dk,dv] or
     None; cu_seqlens int32 [N+1] or None (then ``n_seq`` equal sequences, default 1).
-    Returns (o [T,Hv,dv] in v's dtype, S_T fp32 [N,Hv,dk,dv] or None). Tensors must be
-    contiguous CUDA tensors; nothing is converted or copied here.
+    Returns (o [T,Hv,dv] in ``out_dtype`` (or o's dtype when given), S_T fp32 [N,Hv,dk,dv] or
+    None). Tensors must be contiguous CUDA tensors; nothing is converted or copied here.
     """
     lib = load_library()
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
-    shape = make_shape(q, v, n)
+    if o is not None:
+        out_dtype = o.dtype
+    shape = make_shape(q, v, n, out_dtype)
     T, h_v, dv = v.shape
     if o is None:
-        o = torch.empty((T, h_v, dv), dtype=v.dtype, device=v.device)
+        o = torch.empty((T, h_v, dv), dtype=out_dtype, device=v.device)
     if S_T is None and want_state:
         S_T = torch.empty((n, h_v, q.shape[2], dv), dtype=torch.float32, device=v.device)
     need = gdn2_chunk_fwd_workspace_size(shape, cu_seqlens is not None)
@@ -121,13 +125,15 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=Non
     return o, S_T
 
 
-def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None):
+def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None, out_dtype=torch.float32):
     """One decode token per sequence: q,k [N,Hqk,dk]; v,w [N,Hv,dv]; log_alpha, b [N,Hv,dk];
-    S fp32 [N,Hv,dk,dv] updated in place. Returns o [N,Hv,dv]."""
+    S fp32 [N,Hv,dk,dv] updated in place. Returns o [N,Hv,dv] in ``out_dtype``."""
     lib = load_library()
-    shape = make_shape(q, v, q.shape[0])
+    if o is not None:
+        out_dtype = o.dtype
+    shape = make_shape(q, v, q.shape[0], out_dtype)
     if o is None:
-        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
     _check(lib.gdn2_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                                 _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream_handle(stream)))
     return o

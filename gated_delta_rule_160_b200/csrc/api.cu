@@ -49,6 +49,8 @@ gdn2_status check_shape(const gdn2_shape* sh) {
     if (sh->h_v > 65535) return fail(GDN2_ERR_UNSUPPORTED, "h_v = %d above 65535", sh->h_v);
     if (sh->dtype != GDN2_F32 && sh->dtype != GDN2_BF16)
         return fail(GDN2_ERR_INVALID_ARG, "unknown dtype %d", (int)sh->dtype);
+    if (sh->o_dtype != GDN2_F32 && sh->o_dtype != GDN2_BF16)
+        return fail(GDN2_ERR_INVALID_ARG, "unknown o_dtype %d", (int)sh->o_dtype);
     if ((sh->dk != 64 && sh->dk != 128) || (sh->dv != 64 && sh->dv != 128))
         return fail(GDN2_ERR_UNSUPPORTED, "dk = %d, dv = %d: only 64 and 128 are supported", sh->dk, sh->dv);
     return GDN2_OK;
@@ -140,7 +142,7 @@ gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k
         if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "order kernel: %s", cudaGetErrorString(e));
         p.order = order;
     }
-    cudaError_t e = launch_recurrent(p, shape->dtype, s);
+    cudaError_t e = launch_recurrent(p, shape->dtype, shape->o_dtype, s);
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }
@@ -162,7 +164,7 @@ gdn2_status gdn2_decode_step(const gdn2_shape* shape, const void* q, const void*
     st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
     if (st != GDN2_OK) return st;
     Params p = make_params(shape, q, k, v, log_alpha, b, w, nullptr, nullptr, o, S);
-    cudaError_t e = launch_decode(p, shape->dtype, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_decode(p, shape->dtype, shape->o_dtype, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -21,7 +21,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename T>
+template <int DK, int DV, typename T, typename TO>
 __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     constexpr int TPR = DV / 4;          // threads per state row
     constexpr int RG = kThreads / TPR;   // row groups
@@ -109,30 +109,33 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     }
     if (rg == 0) {
         const float qe = dots[0], qk = dots[1];
-        T* o = static_cast<T*>(p.o) + tv * DV + 4 * cg;
-        o[0] = from_f32<T>(pq.x - qe * r.x + qk * x.x);
-        o[1] = from_f32<T>(pq.y - qe * r.y + qk * x.y);
-        o[2] = from_f32<T>(pq.z - qe * r.z + qk * x.z);
-        o[3] = from_f32<T>(pq.w - qe * r.w + qk * x.w);
+        TO* o = static_cast<TO*>(p.o) + tv * DV + 4 * cg;
+        o[0] = from_f32<TO>(pq.x - qe * r.x + qk * x.x);
+        o[1] = from_f32<TO>(pq.y - qe * r.y + qk * x.y);
+        o[2] = from_f32<TO>(pq.z - qe * r.z + qk * x.z);
+        o[3] = from_f32<TO>(pq.w - qe * r.w + qk * x.w);
     }
 }
 
-template <int DK, int DV, typename T>
+template <int DK, int DV, typename T, typename TO>
 cudaError_t launch_dec(const Params& p, cudaStream_t st) {
-    decode_kernel<DK, DV, T><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
+    decode_kernel<DK, DV, T, TO><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, typename TO>
 cudaError_t launch_dec_t(const Params& p, cudaStream_t s) {
-    if (p.dk == 128) return p.dv == 128 ? launch_dec<128, 128, T>(p, s) : launch_dec<128, 64, T>(p, s);
-    return p.dv == 128 ? launch_dec<64, 128, T>(p, s) : launch_dec<64, 64, T>(p, s);
+    if (p.dk == 128) return p.dv == 128 ? launch_dec<128, 128, T, TO>(p, s) : launch_dec<128, 64, T, TO>(p, s);
+    return p.dv == 128 ? launch_dec<64, 128, T, TO>(p, s) : launch_dec<64, 64, T, TO>(p, s);
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const Params& p, gdn2_dtype dt, cudaStream_t s) {
-    return dt == GDN2_F32 ? launch_dec_t<float>(p, s) : launch_dec_t<__nv_bfloat16>(p, s);
+cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s) {
+    if (dt == GDN2_F32)
+        return odt == GDN2_F32 ? launch_dec_t<float, float>(p, s) : launch_dec_t<float, __nv_bfloat16>(p, s);
+    return odt == GDN2_F32 ? launch_dec_t<__nv_bfloat16, float>(p, s)
+                           : launch_dec_t<__nv_bfloat16, __nv_bfloat16>(p, s);
 }
 
 }  // namespace gdn2

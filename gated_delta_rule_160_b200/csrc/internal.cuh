@@ -47,8 +47,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // Launchers (return cudaGetLastError() of the launch).
-cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, cudaStream_t s);
-cudaError_t launch_decode(const Params& p, gdn2_dtype dt, cudaStream_t s);
+cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s);
+cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s);
 cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s);
 
 }  // namespace gdn2

@@ -33,7 +33,7 @@ struct RecSmem {
     float red[2][2][kSplit][kCols];  // [token parity][r | p][warp][column]
 };
 
-template <int DK, typename T>
+template <int DK, typename T, typename TO>
 __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
     __shared__ RecSmem<DK> sm;
     constexpr int RPT = DK / kSplit;
@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
     const T* vp = static_cast<const T*>(p.v);
     const T* bp = static_cast<const T*>(p.b);
     const T* wp = static_cast<const T*>(p.w);
-    T* op = static_cast<T*>(p.o);
+    TO* op = static_cast<TO*>(p.o);
 
     for (int base = t0; base < t1; base += kStage) {
         const int nt = min(kStage, t1 - base);
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
                 s[i] = fmaf(sm.k[tt][row0 + i], x, fmaf(-sm.e[tt][row0 + i], r, s[i]));
             if (warp == (tt % kSplit)) {
                 const float o = pq - sm.qe[tt] * r + sm.qk[tt] * x;
-                op[((size_t)(base + tt) * p.h_v + h) * dv + col] = from_f32<T>(o);
+                op[((size_t)(base + tt) * p.h_v + h) * dv + col] = from_f32<TO>(o);
             }
         }
     }
@@ -137,18 +137,25 @@ __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
     }
 }
 
-template <int DK, typename T>
+template <int DK, typename T, typename TO>
 cudaError_t launch_rec(const Params& p, cudaStream_t st) {
     dim3 grid(p.dv / kCols, p.h_v, p.n_seq);
-    recurrent_kernel<DK, T><<<grid, kCols * kSplit, 0, st>>>(p);
+    recurrent_kernel<DK, T, TO><<<grid, kCols * kSplit, 0, st>>>(p);
     return cudaGetLastError();
+}
+
+template <typename T, typename TO>
+cudaError_t launch_rec_dk(const Params& p, cudaStream_t s) {
+    return p.dk == 128 ? launch_rec<128, T, TO>(p, s) : launch_rec<64, T, TO>(p, s);
 }
 
 }  // namespace
 
-cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, cudaStream_t s) {
-    if (dt == GDN2_F32) return p.dk == 128 ? launch_rec<128, float>(p, s) : launch_rec<64, float>(p, s);
-    return p.dk == 128 ? launch_rec<128, __nv_bfloat16>(p, s) : launch_rec<64, __nv_bfloat16>(p, s);
+cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s) {
+    if (dt == GDN2_F32)
+        return odt == GDN2_F32 ? launch_rec_dk<float, float>(p, s) : launch_rec_dk<float, __nv_bfloat16>(p, s);
+    return odt == GDN2_F32 ? launch_rec_dk<__nv_bfloat16, float>(p, s)
+                           : launch_rec_dk<__nv_bfloat16, __nv_bfloat16>(p, s);
 }
 
 }  // namespace gdn2

@@ -20,12 +20,16 @@
  *
  * Layouts (row-major, innermost index last, every tensor contiguous):
  *   q, k        [T_total, h_qk, dk]   dtype
- *   v, w, o     [T_total, h_v,  dv]   dtype (o is written in the dtype of v)
+ *   v, w        [T_total, h_v,  dv]   dtype
+ *   o           [T_total, h_v,  dv]   o_dtype
  *   log_alpha   [T_total, h_v,  dk]   float32
  *   b           [T_total, h_v,  dk]   dtype
  *   S0, S_T, S  [n_seq, h_v, dk, dv]  float32 (dv contiguous)
  *   cu_seqlens  [n_seq + 1] int32     packed sequence offsets (0, ..., T_total)
- * dtype GDN2_BF16 means bfloat16; GDN2_F32 means float32 for q, k, v, b, w and o.
+ * dtype GDN2_BF16 means bfloat16, GDN2_F32 float32. o_dtype is chosen separately: a bf16
+ * output carries a rounding error of up to 2^-8 |o| per element, which for these
+ * recurrences (max|o| / rms(o) of 10 to 15) alone exceeds 2e-2 of rms(o); GDN2_F32 output
+ * keeps the result within the kernels' arithmetic error.
  * Value head h reads query/key head h / (h_v / h_qk).
  *
  * Ownership: every tensor pointer is a device pointer owned by the caller and must stay
@@ -75,7 +79,8 @@ typedef struct {
     int h_v;          /* value heads (a multiple of h_qk) */
     int dk;           /* key channels per head: 64 or 128 */
     int dv;           /* value channels per head: 64 or 128 */
-    gdn2_dtype dtype; /* element type of q, k, v, b, w, o */
+    gdn2_dtype dtype;   /* element type of q, k, v, b, w */
+    gdn2_dtype o_dtype; /* element type of o */
 } gdn2_shape;
 
 /*

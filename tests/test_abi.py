@@ -44,7 +44,7 @@ def test_libraries_share_no_symbols(lib, oracle_mod):
 
 
 def _shape(g, **kw):
-    d = dict(n_seq=1, T_total=64, h_qk=1, h_v=1, dk=64, dv=64, dtype=g.GDN2_BF16)
+    d = dict(n_seq=1, T_total=64, h_qk=1, h_v=1, dk=64, dv=64, dtype=g.GDN2_BF16, o_dtype=g.GDN2_F32)
     d.update(kw)
     return g.Shape(**d)
 
@@ -64,6 +64,7 @@ def test_rejects_before_device_work(lib):
     assert _call_chunk(g, lib, _shape(g, h_qk=3, h_v=4)) == 1
     assert _call_chunk(g, lib, _shape(g, n_seq=0)) == 1
     assert _call_chunk(g, lib, _shape(g, dtype=7)) == 1
+    assert _call_chunk(g, lib, _shape(g, o_dtype=5)) == 1
     assert _call_chunk(g, lib, _shape(g)) == 1  # NULL tensors with T_total > 0
     assert b"q is NULL" in lib.gdn2_last_error_string()
     assert _call_chunk(g, lib, _shape(g), ptr=0x1008) == 1  # misaligned

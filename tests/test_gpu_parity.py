@@ -91,6 +91,23 @@ def test_fp32_dk64_dv128_and_no_state_outputs(g, oracle_mod):
     assert st is None and o.shape == d["v"].shape
 
 
+def test_bf16_output_within_one_rounding(g, oracle_mod):
+    """With a bf16 output each element carries at most one rounding (2^-8 relative) on top of
+    the kernel's error: |o - o_ref| <= 2^-8 |o_ref| + 2e-2 rms(o_ref)."""
+    wl = W.WORKLOADS["prefill_b8_h16_t4096"]
+    d = W.prefill_inputs(wl, "cuda", n_seq=2, T=200)
+    for key in ("q", "k", "v", "log_alpha", "b", "w"):
+        d[key] = d[key][:, :2].contiguous()
+    o, _ = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], n_seq=2,
+                            out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    o_ref, _ = oracle_mod.fwd_ref(*(d[k_].cpu() for k_ in ("q", "k", "v", "log_alpha", "b", "w")), n_seq=2)
+    rms = float(np.sqrt(np.mean(o_ref ** 2)))
+    excess = np.abs(o.double().cpu().numpy() - o_ref) - 2.0 ** -8 * np.abs(o_ref)
+    assert excess.max() / rms <= 2e-2
+
+
 def test_empty_input(g):
     d = W.token_inputs(0, 2, 2, 64, 64, torch.bfloat16, "cuda", seed=1)
     S0 = W.state_input(3, 2, 64, 64, 0.1, "cuda", seed=1)
