@@ -142,7 +142,8 @@ gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k
         if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "order kernel: %s", cudaGetErrorString(e));
         p.order = order;
     }
-    cudaError_t e = launch_recurrent(p, shape->dtype, shape->o_dtype, s);
+    cudaError_t e = chunk_tc_supported(p, shape->dtype) ? launch_chunk_tc(p, shape->o_dtype, s)
+                                                        : launch_recurrent(p, shape->dtype, shape->o_dtype, s);
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk kernel launch: %s", cudaGetErrorString(e));
     return ok();
 }

@@ -1,0 +1,623 @@
+// chunk_tc.cu -- chunkwise-parallel prefill on the tcgen05 tensor cores (bf16 inputs,
+// dk = dv = 128, chunks of C = 64 tokens). One CTA of 256 threads owns one (sequence,
+// value head) and walks its chunks in order; the fp32 state lives in tensor memory.
+//
+// Chunk algebra (per chunk, state S on entry; e = b(.)k, x = w(.)v, G = inclusive cumsum
+// of log_alpha over the chunk, per key channel). Every decayed operand is taken relative
+// to a per-channel reference Gref = (G_first + G_last) / 2, so that the factors
+// exp(+-(G - Gref)) stay within about e^+-(half the chunk's decay):
+//   Kh = K exp(G-Gref)   Qh = Q exp(G-Gref)   Kb = K exp(Gref-G)   Eb = E exp(Gref-G)
+//   Gram:  B_ij = Kh_i.Kb_j (j<i)  A_ij = Kh_i.Eb_j (j<i)  P_ij = Qh_i.Kb_j (j<=i)
+//          Qm_ij = Qh_i.Eb_j (j<=i)
+//   T = (I + A)^-1                                  (the gated UT transform)
+//   Y = Kh Sref + B X,  R = T Y                     (key reads of the decayed old state)
+//   O = Qh Sref + P X - Qm R                        (query reads of the updated state)
+//   U = Sref + Kb^T X - Eb^T R,   S' = exp(G_last - Gref) (.) U
+// with Sref = exp(Gref) (.) S. Everything runs transposed (value channel m = row = tensor
+// memory lane) so that every MMA has M = 128.
+//
+// Precision: bf16 operands round to 8 significant bits, and the outputs of this
+// recurrence have max|o| / rms(o) of 10 to 15, so one rounding on a dominant term costs
+// more than the 2e-2 * rms(o) error budget. The terms that carry the output and the
+// state -- P (query/key Gram block), P X, Qh Sref and Kb^T X -- are therefore computed
+// with operands split into bf16 hi + lo parts (three MMAs: hi*hi + lo*hi + hi*lo, about
+// 16 significant bits); the erase path (A, B, Qm, T, Y, R) stays in plain bf16.
+//
+// Phases per chunk (all 256 threads take part in each; thread t serves tensor-memory lane
+// t % 128 and column half t / 128):
+//   1 prep    load the chunk, cumsum log-decays, write the operand tiles
+//   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63)
+//   3 Gram epilogue + fp32 blocked triangular solve for T
+//   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
+//   5 state epilogue: U <- f (.) U, Sref^T hi/lo tiles
+//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh cross term)
+//   7 Y tile  8 MMA R^T = Y^T T^T  9 -R tile  10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
+//   11 o epilogue (fp32 or bf16 stores)
+// The next chunk's rows are prefetched into L2 while the current one is processed.
+#include "internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace gdn2 {
+namespace {
+
+using namespace tc;
+
+constexpr int CH = 64;   // chunk length
+constexpr int D = 128;   // dk = dv
+constexpr int NT = 256;  // threads per CTA
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
+
+// ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
+// row groups outermost (LBO = 128 B, SBO = 2048 B): element (row r, channel c) at
+//   (r/8)*2048 + (c/8)*128 + (r%8)*16 + (c%8)*2.
+constexpr uint32_t kTile = CH * D * 2;   // 16384
+constexpr uint32_t OFF_KH = 0;           // Kh      } rows 0..127 of the Gram B operand
+constexpr uint32_t OFF_QH = 1 * kTile;   // Qh hi   }
+constexpr uint32_t OFF_KBH = 2 * kTile;  // Kb hi   } rows 0..127 of the Gram A operand
+constexpr uint32_t OFF_E = 3 * kTile;    // Eb      }
+constexpr uint32_t OFF_KBL = 4 * kTile;  // Kb lo   (rows 64..127 of its operand are masked out)
+constexpr uint32_t OFF_XH = 5 * kTile;   // X hi
+constexpr uint32_t OFF_XL = 6 * kTile;   // X lo
+constexpr uint32_t OFF_QL = 7 * kTile;   // Qh lo
+// [64][64] bf16 tiles. MN-major B operands B[n=i][k=j] written by the Gram epilogue:
+//   (i/8)*1024 + (j/8)*128 + (j%8)*16 + (i%8)*2     (SBO = 1024, LBO = 128)
+constexpr uint32_t kSmall = CH * CH * 2;  // 8192
+constexpr uint32_t OFF_QM = 8 * kTile;     // Qm
+constexpr uint32_t OFF_T = OFF_QM + kSmall;  // T, K-major [i][j]: (j/8)*1024 + (i/8)*128 + (i%8)*16 + (j%8)*2
+constexpr uint32_t OFF_REG = OFF_T + kSmall;  // 64 KB reused by phases 3 / 5-6 / 7-10
+constexpr uint32_t OFF_B = OFF_REG;             // B   } [B; P hi] is one 128-row operand
+constexpr uint32_t OFF_PH = OFF_REG + kSmall;   // P hi}
+constexpr uint32_t OFF_PL = OFF_REG + 2 * kSmall;
+constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][65]
+constexpr uint32_t OFF_WT = OFF_WA + 64 * 65 * 4;     // fp32 T [64][65]
+constexpr uint32_t OFF_WM = OFF_WT + 64 * 65 * 4;     // fp32 scratch [3][16][17]
+// Row-per-lane tiles [m][k] written by epilogues, K-major, K groups outermost:
+//   (k/8)*2048 + (m/8)*128 + (m%8)*16 + (k%8)*2     (LBO = 2048, SBO = 128)
+constexpr uint32_t OFF_SH = OFF_REG;              // Sref^T hi [128][128]
+constexpr uint32_t OFF_SL = OFF_REG + 2 * kTile;  // Sref^T lo
+constexpr uint32_t OFF_Y = OFF_REG;               // Y^T [128][64]
+constexpr uint32_t OFF_R = OFF_REG + kTile;       // -R^T [128][64]
+constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128]
+constexpr uint32_t OFF_MBAR = OFF_SCAL + 4 * 128 * 4;
+constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
+constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
+static_assert(OFF_WM + 3 * 16 * 17 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// ---- tensor memory columns
+constexpr uint32_t TM_G = 0;     // Gram (transposed): lanes [Kb j ; Eb j], cols [Kh i ; Qh i]
+constexpr uint32_t TM_D1 = 128;  // [Y^T | O^T]
+constexpr uint32_t TM_R = 256;   // R^T
+constexpr uint32_t TM_U = 384;   // state, lanes m (value channel), cols c (key channel)
+
+enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45 };
+
+__device__ unsigned int g_tc_fault = 0;
+
+__device__ __forceinline__ uint32_t off_rowmajor(int r, int c) {  // prep tiles, 128 channels
+    return (uint32_t)((r >> 3) * 2048 + (c >> 3) * 128 + (r & 7) * 16 + (c & 7) * 2);
+}
+__device__ __forceinline__ uint32_t off_lane_k(int m, int k) {     // epilogue tiles, 128 lanes
+    return (uint32_t)((k >> 3) * 2048 + (m >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// 4 consecutive bf16 values (8 bytes) widened to fp32.
+__device__ __forceinline__ void unpack4_bf16(uint2 u, float (&f)[4]) {
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x), b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    f[0] = __low2float(a);
+    f[1] = __high2float(a);
+    f[2] = __low2float(b);
+    f[3] = __high2float(b);
+}
+
+__device__ __forceinline__ void store4_bf16(uint8_t* smem, uint32_t off, const float (&f)[4]) {
+    *reinterpret_cast<uint2*>(smem + off) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+}
+
+// 8 fp32 values as 8 bf16 in one 16-byte shared store.
+__device__ __forceinline__ void store8_bf16(uint8_t* smem, uint32_t off, const float* f) {
+    *reinterpret_cast<uint4*>(smem + off) =
+        make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+}
+
+template <typename TO>
+__global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int L = tid & 127;   // tensor-memory lane served by this thread
+    const int hf = tid >> 7;   // column half
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
+    float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] g2ref, [256..511] g2last
+    float* WA = reinterpret_cast<float*>(smem + OFF_WA);
+    float* WT = reinterpret_cast<float*>(smem + OFF_WT);
+    float* WM = reinterpret_cast<float*>(smem + OFF_WM);
+    const uint32_t mbar0 = sbase + OFF_MBAR;
+    auto mbar = [&](int i) { return mbar0 + 8u * (uint32_t)i; };
+
+    const int item = blockIdx.x;
+    const int n = p.order ? p.order[item / p.h_v] : item / p.h_v;
+    const int h = item % p.h_v;
+    const int g = h / (p.h_v / p.h_qk);
+    int t0, t1;
+    seq_bounds(p, n, t0, t1);
+    const int nchunks = (t1 - t0 + CH - 1) / CH;
+    const size_t soff = ((size_t)n * p.h_v + h) * D * D;
+
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(p.q);
+    const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(p.k);
+    const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(p.v);
+    const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
+    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(p.w);
+    TO* op = static_cast<TO*>(p.o);
+
+    if (nchunks == 0) {  // empty sequence: S_T = S0
+        if (p.S_T)
+            for (int i = tid; i < D * D; i += NT) p.S_T[soff + i] = p.S0 ? p.S0[soff + i] : 0.f;
+        return;
+    }
+
+    if (tid == 0) {
+        for (int i = 0; i < 5; ++i) mbar_init(mbar(i), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
+    bool fault = false;
+
+    // prep mapping: warp w owns channels [16w, 16w+16); lane = (channel quad, token in block)
+    const int tl = lane & 7;
+    const int c0 = 16 * warp + 4 * (lane >> 3);
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int tc0 = t0 + ci * CH;
+        const int nvalid = min(CH, t1 - tc0);
+        const int buf = ci & 1;
+        const uint32_t par = (uint32_t)(ci & 1);
+
+        // ------------------------------------------------------------ 1. prep
+        {
+            // every load of the chunk is issued before any arithmetic (8 passes x 6 loads in flight)
+            float4 la[8];
+            uint2 kq[8], qq[8], bq[8], vq[8], wq[8];
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                const bool valid = i < nvalid;
+                const size_t tq = ((size_t)(tc0 + i) * p.h_qk + g) * D + c0;
+                const size_t tv = ((size_t)(tc0 + i) * p.h_v + h) * D + c0;
+                const uint2 z = make_uint2(0u, 0u);
+                la[pss] = valid ? *reinterpret_cast<const float4*>(p.log_alpha + tv) : make_float4(0.f, 0.f, 0.f, 0.f);
+                kq[pss] = valid ? *reinterpret_cast<const uint2*>(kp + tq) : z;
+                qq[pss] = valid ? *reinterpret_cast<const uint2*>(qp + tq) : z;
+                bq[pss] = valid ? *reinterpret_cast<const uint2*>(bp + tv) : z;
+                vq[pss] = valid ? *reinterpret_cast<const uint2*>(vp + tv) : z;
+                wq[pss] = valid ? *reinterpret_cast<const uint2*>(wp + tv) : z;
+            }
+            float G[8][4];
+            float carry[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                float x[4] = {la[pss].x * kLog2e, la[pss].y * kLog2e, la[pss].z * kLog2e, la[pss].w * kLog2e};
+#pragma unroll
+                for (int dlt = 1; dlt < 8; dlt <<= 1) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float y = __shfl_up_sync(0xffffffffu, x[e], dlt, 8);
+                        if (tl >= dlt) x[e] += y;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    G[pss][e] = x[e] + carry[e];
+                    carry[e] = __shfl_sync(0xffffffffu, G[pss][e], (lane & 24) | 7);
+                }
+            }
+            float gref[4], glast[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float gfirst = __shfl_sync(0xffffffffu, G[0][e], lane & 24);
+                glast[e] = carry[e];
+                gref[e] = 0.5f * (gfirst + glast[e]);
+            }
+            if (tl == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    scal[buf * 128 + c0 + e] = gref[e];
+                    scal[256 + buf * 128 + c0 + e] = glast[e];
+                }
+            }
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                float kf[4], qf[4], bf[4], vf[4], wf[4];
+                unpack4_bf16(kq[pss], kf);
+                unpack4_bf16(qq[pss], qf);
+                unpack4_bf16(bq[pss], bf);
+                unpack4_bf16(vq[pss], vf);
+                unpack4_bf16(wq[pss], wf);
+                float kh[4], qh[4], ql[4], kbh[4], kbl[4], eb[4], xh[4], xl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ge = exp2f(G[pss][e] - gref[e]);
+                    const float gi = exp2f(gref[e] - G[pss][e]);
+                    kh[e] = kf[e] * ge;
+                    const float qv = qf[e] * ge;
+                    qh[e] = bf16_round(qv);
+                    ql[e] = qv - qh[e];
+                    const float kb = kf[e] * gi;
+                    kbh[e] = bf16_round(kb);
+                    kbl[e] = kb - kbh[e];
+                    eb[e] = bf[e] * kf[e] * gi;
+                    const float xv = wf[e] * vf[e];
+                    xh[e] = bf16_round(xv);
+                    xl[e] = xv - xh[e];
+                }
+                const uint32_t o = off_rowmajor(i, c0);
+                store4_bf16(smem, OFF_KH + o, kh);
+                store4_bf16(smem, OFF_QH + o, qh);
+                store4_bf16(smem, OFF_QL + o, ql);
+                store4_bf16(smem, OFF_KBH + o, kbh);
+                store4_bf16(smem, OFF_KBL + o, kbl);
+                store4_bf16(smem, OFF_E + o, eb);
+                store4_bf16(smem, OFF_XH + o, xh);
+                store4_bf16(smem, OFF_XL + o, xl);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ------------------------------------------------------------ 2. Gram MMAs
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id128 = idesc_bf16(128, 128, false, false);
+            const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t kofs = ks * 256;
+                mma_bf16(tmem + TM_G, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
+                         sdesc(sbase + OFF_KH + kofs, 128, 2048), id128, ks > 0);
+            }
+            // P cross terms (lanes 0..63 hold Kb rows; lanes 64..127 are masked out)
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint32_t kofs = ks * 256;
+                mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBL + kofs, 128, 2048),
+                         sdesc(sbase + OFF_QH + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
+                mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
+                         sdesc(sbase + OFF_QL + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
+            }
+            mma_commit(mbar(MB_G));
+        } else if (warp == 1 && ci + 1 < nchunks) {
+            // bring the next chunk's rows into L2 while this one is computed
+            const int tn = tc0 + CH;
+            const int nn = min(CH, t1 - tn);
+            for (int r = lane; r < nn; r += 32) {
+                const size_t tq = ((size_t)(tn + r) * p.h_qk + g) * D;
+                const size_t tv = ((size_t)(tn + r) * p.h_v + h) * D;
+                prefetch_l2(qp + tq, D * 2);
+                prefetch_l2(kp + tq, D * 2);
+                prefetch_l2(vp + tv, D * 2);
+                prefetch_l2(wp + tv, D * 2);
+                prefetch_l2(bp + tv, D * 2);
+                prefetch_l2(p.log_alpha + tv, D * 4);
+            }
+        }
+        fault |= !mbar_wait(mbar(MB_G), par, kWaitNs);
+        if (__syncthreads_or(fault)) { fault = true; break; }
+        tc_fence_after();
+
+        // ------------------------------------------------------------ 3. Gram epilogue
+        {
+            float v0[32], v1[32];
+            tmem_ld32(tmem + lane_bits + TM_G + 64 * hf, v0);
+            tmem_ld32(tmem + lane_bits + TM_G + 64 * hf + 32, v1);
+            tmem_wait_ld();
+            const int j = L & 63;
+            auto val = [&](int i) { return i < 32 ? v0[i] : v1[i - 32]; };
+            if (L < 64 && hf == 0) {  // B_ij, j < i
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = (8 * q8 + e > j) ? val(8 * q8 + e) : 0.f;
+                    store8_bf16(smem, OFF_B + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
+                }
+            } else if (L < 64) {  // P_ij, j <= i, split hi / lo
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    float fh[8], fl[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
+                        fh[e] = bf16_round(x);
+                        fl[e] = x - fh[e];
+                    }
+                    const uint32_t o = q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16;
+                    store8_bf16(smem, OFF_PH + o, fh);
+                    store8_bf16(smem, OFF_PL + o, fl);
+                }
+            } else if (hf == 0) {  // A_ij, j < i, fp32 for the solve
+#pragma unroll
+                for (int i = 0; i < 64; ++i) WA[i * 65 + j] = (i > j) ? val(i) : 0.f;
+            } else {  // Qm_ij, j <= i
+#pragma unroll
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
+                    store8_bf16(smem, OFF_QM + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
+                }
+            }
+        }
+        __syncthreads();
+        // T = (I + A)^-1 by 16 x 16 blocks. Diagonal blocks: column-wise forward
+        // substitution; off-diagonal blocks by distance d: T_IJ = -T_II sum_L A_IL T_LJ.
+        if (tid < 64) {
+            const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float s = 0.f;
+#pragma unroll
+                for (int l = 0; l < r; ++l) s += (l >= jj) ? WA[(16 * bI + r) * 65 + 16 * bI + l] * x[l] : 0.f;
+                x[r] = (r < jj) ? 0.f : (r == jj ? 1.f : -s);
+                WT[(16 * bI + r) * 65 + col] = x[r];
+            }
+        } else {
+            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
+                const int r = idx >> 6, c = idx & 63;
+                if ((c >> 4) > (r >> 4)) WT[r * 65 + c] = 0.f;
+            }
+        }
+        __syncthreads();
+        for (int d = 1; d <= 3; ++d) {
+            const int nel = (4 - d) * 256;
+            for (int e = tid; e < nel; e += NT) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
+                float s = 0.f;
+                for (int Lb = J; Lb < I; ++Lb)
+#pragma unroll
+                    for (int l = 0; l < 16; ++l)
+                        s += WA[(16 * I + r) * 65 + 16 * Lb + l] * WT[(16 * Lb + l) * 65 + 16 * J + cc];
+                WM[(J * 16 + r) * 17 + cc] = s;
+            }
+            __syncthreads();
+            for (int e = tid; e < nel; e += NT) {
+                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
+                float s = 0.f;
+#pragma unroll
+                for (int l = 0; l < 16; ++l)
+                    if (l <= r) s += WT[(16 * I + r) * 65 + 16 * I + l] * WM[(J * 16 + l) * 17 + cc];
+                WT[(16 * I + r) * 65 + 16 * J + cc] = -s;
+            }
+            __syncthreads();
+        }
+        for (int idx = tid; idx < 512; idx += NT) {  // T as a K-major bf16 B operand [i][j]
+            const int i = idx & 63, jg = idx >> 6;
+            store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * 65 + 8 * jg]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------------------------------------ 4. D1 = X^T [B;P]^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id128 = idesc_bf16(128, 128, true, true);
+            const uint32_t id64 = idesc_bf16(128, 64, true, true);
+#pragma unroll
+            for (int ks = 0; ks < CH / 16; ++ks) {
+                const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
+                const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
+                mma_bf16(tmem + TM_D1, xh, sdesc(sbase + OFF_B + ks * 256, 128, 1024), id128, ks > 0);
+                mma_bf16(tmem + TM_D1 + 64, xl, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
+                mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PL + ks * 256, 128, 1024), id64, 1u);
+            }
+            mma_commit(mbar(MB_2B));
+        }
+        fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
+        if (__syncthreads_or(fault)) { fault = true; break; }
+        tc_fence_after();
+
+        // ------------------------------------------------------------ 5. state epilogue
+        {
+            const float* gref_cur = scal + buf * 128;
+            const float* gref_prev = scal + (buf ^ 1) * 128;
+            const float* glast_prev = scal + 256 + (buf ^ 1) * 128;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int cb = 64 * hf + 32 * part;
+                float u[32];
+                if (ci == 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = cb + e;
+                        const float s0 = p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f;
+                        u[e] = s0 * exp2f(gref_cur[c]);
+                    }
+                } else {
+                    tmem_ld32(tmem + lane_bits + TM_U + cb, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = cb + e;
+                        u[e] *= exp2f(glast_prev[c] - gref_prev[c] + gref_cur[c]);
+                    }
+                }
+                tmem_st32(tmem + lane_bits + TM_U + cb, u);
+#pragma unroll
+                for (int e8 = 0; e8 < 4; ++e8) {
+                    float fh[8], fl[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        fh[e] = bf16_round(u[8 * e8 + e]);
+                        fl[e] = u[8 * e8 + e] - fh[e];
+                    }
+                    const uint32_t o = off_lane_k(L, cb + 8 * e8);
+                    store8_bf16(smem, OFF_SH + o, fh);
+                    store8_bf16(smem, OFF_SL + o, fl);
+                }
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------------------------------------ 6. D1 += Sref^T [Kh;Qh]^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id128 = idesc_bf16(128, 128, false, false);
+            const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_SH + ks * 4096, 2048, 128),
+                         sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
+                mma_bf16(tmem + TM_D1 + 64, sdesc(sbase + OFF_SL + ks * 4096, 2048, 128),
+                         sdesc(sbase + OFF_QH + ks * 256, 128, 2048), id64, 1u);
+            }
+            mma_commit(mbar(MB_2A));
+        }
+        fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
+        if (__syncthreads_or(fault)) { fault = true; break; }
+        tc_fence_after();
+
+        // ------------------------------------------------------------ 7. Y^T tile
+        {
+            float y[32];
+            tmem_ld32(tmem + lane_bits + TM_D1 + 32 * hf, y);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_Y + off_lane_k(L, 32 * hf + 8 * e8), &y[8 * e8]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------------------------------------ 8. R^T = Y^T T^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int ks = 0; ks < CH / 16; ++ks)
+                mma_bf16(tmem + TM_R, sdesc(sbase + OFF_Y + ks * 4096, 2048, 128),
+                         sdesc(sbase + OFF_T + ks * 2048, 1024, 128), id64, ks > 0);
+            mma_commit(mbar(MB_3));
+        }
+        fault |= !mbar_wait(mbar(MB_3), par, kWaitNs);
+        if (__syncthreads_or(fault)) { fault = true; break; }
+        tc_fence_after();
+
+        // ------------------------------------------------------------ 9. -R^T tile
+        {
+            float r[32];
+            tmem_ld32(tmem + lane_bits + TM_R + 32 * hf, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = -r[e];
+#pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_R + off_lane_k(L, 32 * hf + 8 * e8), &r[8 * e8]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ------------------------------------------------------------ 10. output and state MMAs
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_o = idesc_bf16(128, 64, false, true);
+            const uint32_t id_xx = idesc_bf16(128, 128, true, true);
+            const uint32_t id_rx = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int ks = 0; ks < CH / 16; ++ks) {
+                const uint64_t rr = sdesc(sbase + OFF_R + ks * 4096, 2048, 128);
+                const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
+                const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
+                mma_bf16(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
+                mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
+                mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
+                mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
+                mma_bf16(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
+            }
+            mma_commit(mbar(MB_45));
+        }
+        fault |= !mbar_wait(mbar(MB_45), par, kWaitNs);
+        if (__syncthreads_or(fault)) { fault = true; break; }
+        tc_fence_after();
+
+        // ------------------------------------------------------------ 11. o
+        {
+            float ov[32];
+            tmem_ld32(tmem + lane_bits + TM_D1 + 64 + 32 * hf, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int i = 32 * hf + e;
+                if (i < nvalid) op[((size_t)(tc0 + i) * p.h_v + h) * D + L] = from_f32<TO>(ov[e]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    if (!fault && p.S_T) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
+        const int buf = (nchunks - 1) & 1;
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int cb = 64 * hf + 32 * part;
+            float u[32];
+            tmem_ld32(tmem + lane_bits + TM_U + cb, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int c = cb + e;
+                p.S_T[soff + (size_t)c * D + L] = u[e] * exp2f(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
+            }
+        }
+    }
+    if (fault && tid == 0) atomicOr(&g_tc_fault, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <typename TO>
+cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
+    // set on every launch: the attribute is per device and the call costs microseconds
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    chunk_tc_kernel<TO><<<p.n_seq * p.h_v, NT, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_tc_supported(const Params& p, gdn2_dtype dt) {
+    return dt == GDN2_BF16 && p.dk == D && p.dv == D;
+}
+
+cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s) {
+    return odt == GDN2_F32 ? launch_tc_t<float>(p, s) : launch_tc_t<__nv_bfloat16>(p, s);
+}
+
+cudaError_t read_tc_fault(unsigned int* out) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_fault, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_tc_fault, &zero, sizeof(unsigned int));
+}
+
+}  // namespace gdn2

@@ -50,5 +50,8 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s);
 cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s);
 cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s);
+bool chunk_tc_supported(const Params& p, gdn2_dtype dt);
+cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);
+cudaError_t read_tc_fault(unsigned int* out);
 
 }  // namespace gdn2
