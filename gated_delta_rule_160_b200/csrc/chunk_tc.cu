@@ -19,18 +19,19 @@
 // Precision: bf16 operands round to 8 significant bits, and the outputs of this
 // recurrence have max|o| / rms(o) of 10 to 15, so one rounding on a dominant term costs
 // more than the 2e-2 * rms(o) error budget. The terms that carry the output and the
-// state -- P (query/key Gram block), P X, Qh Sref and Kb^T X -- are therefore computed
-// with operands split into bf16 hi + lo parts (three MMAs: hi*hi + lo*hi + hi*lo, about
-// 16 significant bits); the erase path (A, B, Qm, T, Y, R) stays in plain bf16.
+// state -- P (query/key Gram block), P X and Kb^T X -- are therefore computed with both
+// operands split into bf16 hi + lo parts (three MMAs: hi*hi + lo*hi + hi*lo, about 16
+// significant bits); Qh Sref splits Qh only (Qh_hi Sref + Qh_lo Sref); the erase path
+// (A, B, Qm, T, Y, R) stays in plain bf16.
 //
 // Phases per chunk (all 256 threads take part in each; thread t serves tensor-memory lane
 // t % 128 and column half t / 128):
 //   1 prep    load the chunk, cumsum log-decays, write the operand tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63)
-//   3 Gram epilogue + fp32 blocked triangular solve for T
+//   3 Gram epilogue + fp32 blocked triangular solve for T (16 -> 32 -> 64)
 //   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
-//   5 state epilogue: U <- f (.) U, Sref^T hi/lo tiles
-//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh cross term)
+//   5 state epilogue: U <- f (.) U, Sref^T tile
+//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term)
 //   7 Y tile  8 MMA R^T = Y^T T^T  9 -R tile  10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
 //   11 o epilogue (fp32 or bf16 stores)
 // The next chunk's rows are prefetched into L2 while the current one is processed.
@@ -71,18 +72,17 @@ constexpr uint32_t OFF_PH = OFF_REG + kSmall;   // P hi}
 constexpr uint32_t OFF_PL = OFF_REG + 2 * kSmall;
 constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][65]
 constexpr uint32_t OFF_WT = OFF_WA + 64 * 65 * 4;     // fp32 T [64][65]
-constexpr uint32_t OFF_WM = OFF_WT + 64 * 65 * 4;     // fp32 scratch [3][16][17]
+constexpr uint32_t OFF_WM = OFF_WT + 64 * 65 * 4;     // fp32 scratch [32][33]
 // Row-per-lane tiles [m][k] written by epilogues, K-major, K groups outermost:
 //   (k/8)*2048 + (m/8)*128 + (m%8)*16 + (k%8)*2     (LBO = 2048, SBO = 128)
-constexpr uint32_t OFF_SH = OFF_REG;              // Sref^T hi [128][128]
-constexpr uint32_t OFF_SL = OFF_REG + 2 * kTile;  // Sref^T lo
+constexpr uint32_t OFF_SH = OFF_REG;              // Sref^T (bf16) [128][128]
 constexpr uint32_t OFF_Y = OFF_REG;               // Y^T [128][64]
 constexpr uint32_t OFF_R = OFF_REG + kTile;       // -R^T [128][64]
-constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128]
-constexpr uint32_t OFF_MBAR = OFF_SCAL + 4 * 128 * 4;
+constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128], f[128]
+constexpr uint32_t OFF_MBAR = OFF_SCAL + 5 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
-static_assert(OFF_WM + 3 * 16 * 17 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
+static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- tensor memory columns
@@ -107,6 +107,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// Split 2 fp32 values into bf16 hi (packed) and bf16 lo = x - hi (packed): hi + lo carries
+// about 16 significant bits.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    hi = pack_bf16(a, b);
+    const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xffff0000u);
+    lo = pack_bf16(a - ha, b - hb);
+}
 
 // 4 consecutive bf16 values (8 bytes) widened to fp32.
 __device__ __forceinline__ void unpack4_bf16(uint2 u, float (&f)[4]) {
@@ -136,6 +144,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
     float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] g2ref, [256..511] g2last
+    float* fscal = scal + 512;                                  // [128] state frame factors
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
     float* WT = reinterpret_cast<float*>(smem + OFF_WT);
     float* WM = reinterpret_cast<float*>(smem + OFF_WM);
@@ -204,6 +213,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
                 vq[pss] = valid ? *reinterpret_cast<const uint2*>(vp + tv) : z;
                 wq[pss] = valid ? *reinterpret_cast<const uint2*>(wp + tv) : z;
             }
+            if (ci + 1 < nchunks) {
+                // bring the next chunk's rows into L2 (14 lines of 128 B per token) while
+                // this one is processed; one line per instruction keeps the issue cheap
+                const int tn = tc0 + CH;
+                const int nn = min(CH, t1 - tn);
+                for (int idx = tid; idx < nn * 14; idx += NT) {
+                    const int r = idx / 14, ln = idx % 14;
+                    const size_t tq = ((size_t)(tn + r) * p.h_qk + g) * D;
+                    const size_t tv = ((size_t)(tn + r) * p.h_v + h) * D;
+                    const char* a;
+                    if (ln < 2) a = reinterpret_cast<const char*>(qp + tq) + 128 * ln;
+                    else if (ln < 4) a = reinterpret_cast<const char*>(kp + tq) + 128 * (ln - 2);
+                    else if (ln < 6) a = reinterpret_cast<const char*>(vp + tv) + 128 * (ln - 4);
+                    else if (ln < 8) a = reinterpret_cast<const char*>(wp + tv) + 128 * (ln - 6);
+                    else if (ln < 10) a = reinterpret_cast<const char*>(bp + tv) + 128 * (ln - 8);
+                    else a = reinterpret_cast<const char*>(p.log_alpha + tv) + 128 * (ln - 10);
+                    prefetch_line_l2(a);
+                }
+            }
             float G[8][4];
             float carry[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -233,8 +261,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
             if (tl == 0) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    scal[buf * 128 + c0 + e] = gref[e];
-                    scal[256 + buf * 128 + c0 + e] = glast[e];
+                    const int c = c0 + e;
+                    // factor taking the state from the previous chunk's reference frame (or
+                    // S0) into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
+                    fscal[c] = ci == 0 ? exp2f(gref[e])
+                                       : exp2f(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref[e]);
+                    scal[buf * 128 + c] = gref[e];
+                    scal[256 + buf * 128 + c] = glast[e];
                 }
             }
 #pragma unroll
@@ -246,32 +279,33 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
                 unpack4_bf16(bq[pss], bf);
                 unpack4_bf16(vq[pss], vf);
                 unpack4_bf16(wq[pss], wf);
-                float kh[4], qh[4], ql[4], kbh[4], kbl[4], eb[4], xh[4], xl[4];
+                float kh[4], qv[4], kb[4], eb[4], xv[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float ge = exp2f(G[pss][e] - gref[e]);
                     const float gi = exp2f(gref[e] - G[pss][e]);
                     kh[e] = kf[e] * ge;
-                    const float qv = qf[e] * ge;
-                    qh[e] = bf16_round(qv);
-                    ql[e] = qv - qh[e];
-                    const float kb = kf[e] * gi;
-                    kbh[e] = bf16_round(kb);
-                    kbl[e] = kb - kbh[e];
+                    qv[e] = qf[e] * ge;
+                    kb[e] = kf[e] * gi;
                     eb[e] = bf[e] * kf[e] * gi;
-                    const float xv = wf[e] * vf[e];
-                    xh[e] = bf16_round(xv);
-                    xl[e] = xv - xh[e];
+                    xv[e] = wf[e] * vf[e];
                 }
+                uint2 qh, ql, kbh, kbl, xh, xl;
+                split2(qv[0], qv[1], qh.x, ql.x);
+                split2(qv[2], qv[3], qh.y, ql.y);
+                split2(kb[0], kb[1], kbh.x, kbl.x);
+                split2(kb[2], kb[3], kbh.y, kbl.y);
+                split2(xv[0], xv[1], xh.x, xl.x);
+                split2(xv[2], xv[3], xh.y, xl.y);
                 const uint32_t o = off_rowmajor(i, c0);
                 store4_bf16(smem, OFF_KH + o, kh);
-                store4_bf16(smem, OFF_QH + o, qh);
-                store4_bf16(smem, OFF_QL + o, ql);
-                store4_bf16(smem, OFF_KBH + o, kbh);
-                store4_bf16(smem, OFF_KBL + o, kbl);
                 store4_bf16(smem, OFF_E + o, eb);
-                store4_bf16(smem, OFF_XH + o, xh);
-                store4_bf16(smem, OFF_XL + o, xl);
+                *reinterpret_cast<uint2*>(smem + OFF_QH + o) = qh;
+                *reinterpret_cast<uint2*>(smem + OFF_QL + o) = ql;
+                *reinterpret_cast<uint2*>(smem + OFF_KBH + o) = kbh;
+                *reinterpret_cast<uint2*>(smem + OFF_KBL + o) = kbl;
+                *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
+                *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
             }
         }
         fence_proxy_async_smem();
@@ -298,20 +332,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
                          sdesc(sbase + OFF_QL + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
             }
             mma_commit(mbar(MB_G));
-        } else if (warp == 1 && ci + 1 < nchunks) {
-            // bring the next chunk's rows into L2 while this one is computed
-            const int tn = tc0 + CH;
-            const int nn = min(CH, t1 - tn);
-            for (int r = lane; r < nn; r += 32) {
-                const size_t tq = ((size_t)(tn + r) * p.h_qk + g) * D;
-                const size_t tv = ((size_t)(tn + r) * p.h_v + h) * D;
-                prefetch_l2(qp + tq, D * 2);
-                prefetch_l2(kp + tq, D * 2);
-                prefetch_l2(vp + tv, D * 2);
-                prefetch_l2(wp + tv, D * 2);
-                prefetch_l2(bp + tv, D * 2);
-                prefetch_l2(p.log_alpha + tv, D * 4);
-            }
         }
         fault |= !mbar_wait(mbar(MB_G), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
@@ -336,16 +356,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
             } else if (L < 64) {  // P_ij, j <= i, split hi / lo
 #pragma unroll
                 for (int q8 = 0; q8 < 8; ++q8) {
-                    float fh[8], fl[8];
+                    float x[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float x = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
-                        fh[e] = bf16_round(x);
-                        fl[e] = x - fh[e];
-                    }
+                    for (int e = 0; e < 8; ++e) x[e] = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
+                    uint4 hi, lo;
+                    split2(x[0], x[1], hi.x, lo.x);
+                    split2(x[2], x[3], hi.y, lo.y);
+                    split2(x[4], x[5], hi.z, lo.z);
+                    split2(x[6], x[7], hi.w, lo.w);
                     const uint32_t o = q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16;
-                    store8_bf16(smem, OFF_PH + o, fh);
-                    store8_bf16(smem, OFF_PL + o, fl);
+                    *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
+                    *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
                 }
             } else if (hf == 0) {  // A_ij, j < i, fp32 for the solve
 #pragma unroll
@@ -361,8 +382,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
             }
         }
         __syncthreads();
-        // T = (I + A)^-1 by 16 x 16 blocks. Diagonal blocks: column-wise forward
-        // substitution; off-diagonal blocks by distance d: T_IJ = -T_II sum_L A_IL T_LJ.
+        // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
+        // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
+        // and of 32 into 64 with T_21 = -T_22 (A_21 T_11).
         if (tid < 64) {
             const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
             float x[16];
@@ -381,28 +403,60 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
             }
         }
         __syncthreads();
-        for (int d = 1; d <= 3; ++d) {
-            const int nel = (4 - d) * 256;
-            for (int e = tid; e < nel; e += NT) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-                float s = 0.f;
-                for (int Lb = J; Lb < I; ++Lb)
+        {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
+            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
+            float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-                    for (int l = 0; l < 16; ++l)
-                        s += WA[(16 * I + r) * 65 + 16 * Lb + l] * WT[(16 * Lb + l) * 65 + 16 * J + cc];
-                WM[(J * 16 + r) * 17 + cc] = s;
+            for (int l = 0; l < 16; ++l) {
+                const float t = WT[(base + l) * 65 + base + c];
+                m0 += WA[(base + 16 + r0) * 65 + base + l] * t;
+                m1 += WA[(base + 24 + r0) * 65 + base + l] * t;
             }
-            __syncthreads();
-            for (int e = tid; e < nel; e += NT) {
-                const int J = e >> 8, I = J + d, r = (e >> 4) & 15, cc = e & 15;
-                float s = 0.f;
-#pragma unroll
-                for (int l = 0; l < 16; ++l)
-                    if (l <= r) s += WT[(16 * I + r) * 65 + 16 * I + l] * WM[(J * 16 + l) * 17 + cc];
-                WT[(16 * I + r) * 65 + 16 * J + cc] = -s;
-            }
-            __syncthreads();
+            WM[((tid >> 7) * 16 + r0) * 33 + c] = m0;
+            WM[((tid >> 7) * 16 + r0 + 8) * 33 + c] = m1;
         }
+        __syncthreads();
+        {   // level 2, step 2: T_10 = -T_11 M
+            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
+            const float* Mb = WM + (tid >> 7) * 16 * 33;
+            float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+            for (int l = 0; l < 16; ++l) {
+                const float mv = Mb[l * 33 + c];
+                if (l <= r0) t0 += WT[(base + 16 + r0) * 65 + base + 16 + l] * mv;
+                if (l <= r0 + 8) t1 += WT[(base + 24 + r0) * 65 + base + 16 + l] * mv;
+            }
+            WT[(base + 16 + r0) * 65 + base + c] = -t0;
+            WT[(base + 24 + r0) * 65 + base + c] = -t1;
+        }
+        __syncthreads();
+        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
+            const int c = tid & 31, r0 = tid >> 5;
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int l = 0; l < 32; ++l) {
+                const float t = WT[l * 65 + c];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m[k] += WA[(32 + r0 + 8 * k) * 65 + l] * t;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) WM[(r0 + 8 * k) * 33 + c] = m[k];
+        }
+        __syncthreads();
+        {   // level 3, step 2: T_BA = -T_BB M
+            const int c = tid & 31, r0 = tid >> 5;
+            float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int l = 0; l < 32; ++l) {
+                const float mv = WM[l * 33 + c];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (l <= r0 + 8 * k) t[k] += WT[(32 + r0 + 8 * k) * 65 + 32 + l] * mv;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) WT[(32 + r0 + 8 * k) * 65 + c] = -t[k];
+        }
+        __syncthreads();
         for (int idx = tid; idx < 512; idx += NT) {  // T as a K-major bf16 B operand [i][j]
             const int i = idx & 63, jg = idx >> 6;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * 65 + 8 * jg]);
@@ -432,9 +486,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
 
         // ------------------------------------------------------------ 5. state epilogue
         {
-            const float* gref_cur = scal + buf * 128;
-            const float* gref_prev = scal + (buf ^ 1) * 128;
-            const float* glast_prev = scal + 256 + (buf ^ 1) * 128;
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 const int cb = 64 * hf + 32 * part;
@@ -443,31 +494,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int c = cb + e;
-                        const float s0 = p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f;
-                        u[e] = s0 * exp2f(gref_cur[c]);
+                        u[e] = (p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f) * fscal[c];
                     }
                 } else {
                     tmem_ld32(tmem + lane_bits + TM_U + cb, u);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = cb + e;
-                        u[e] *= exp2f(glast_prev[c] - gref_prev[c] + gref_cur[c]);
-                    }
+                    for (int e = 0; e < 32; ++e) u[e] *= fscal[cb + e];
                 }
                 tmem_st32(tmem + lane_bits + TM_U + cb, u);
 #pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    float fh[8], fl[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        fh[e] = bf16_round(u[8 * e8 + e]);
-                        fl[e] = u[8 * e8 + e] - fh[e];
-                    }
-                    const uint32_t o = off_lane_k(L, cb + 8 * e8);
-                    store8_bf16(smem, OFF_SH + o, fh);
-                    store8_bf16(smem, OFF_SL + o, fl);
-                }
+                for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_SH + off_lane_k(L, cb + 8 * e8), &u[8 * e8]);
             }
             tmem_wait_st();
         }
@@ -484,8 +521,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
             for (int ks = 0; ks < D / 16; ++ks) {
                 mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_SH + ks * 4096, 2048, 128),
                          sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
-                mma_bf16(tmem + TM_D1 + 64, sdesc(sbase + OFF_SL + ks * 4096, 2048, 128),
-                         sdesc(sbase + OFF_QH + ks * 256, 128, 2048), id64, 1u);
+                mma_bf16(tmem + TM_D1 + 64, sdesc(sbase + OFF_SH + ks * 4096, 2048, 128),
+                         sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
             }
             mma_commit(mbar(MB_2A));
         }
