@@ -108,6 +108,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def recorded_traffic(profile_name: str, source_rel: str):
+    """DRAM bytes per launch recorded from an ncu capture summarised in profiles/, or None
+    when the kernel source has changed since the capture (its sha256 prefix differs)."""
+    import hashlib
+    import re
+    try:
+        with open(os.path.join(ROOT, "profiles", profile_name)) as f:
+            text = f.read()
+        with open(os.path.join(ROOT, source_rel), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch=(\S+) kernel_sha256_prefix=(\w+)", text)
+    if not m or m.group(2) != sha or m.group(1) == "null":
+        return None
+    return int(m.group(1))
+
+
 def prefill_bytes(wl, lengths) -> int:
     """Algorithmic bytes of one chunk-forward: every input read once, o and S_T written once;
     q and k are counted once per query/key head (value heads in a group share them)."""
@@ -259,7 +277,9 @@ def main():
     nbytes = prefill_bytes(wl, d["lengths"])
     achieved = nbytes / (kern_ms / 1000.0) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": None,
+                "frac": achieved / hbm,
+                "traffic": recorded_traffic("chunk_tc_prefill_b8_h16_t4096.md",
+                                            "gated_delta_rule_160_b200/csrc/chunk_tc.cu"),
                 "peak_source": f"{peak_src} hbm_gbs", "kernel": "gdn2 chunk-forward",
                 "algorithmic_bytes_per_launch": nbytes}
 
@@ -288,7 +308,9 @@ def main():
               "config": {"workload": DECODE, "n_seq": dwl.n_seq, "heads": dwl.h_v, "dk": dwl.dk,
                          "dv": dwl.dv, "state_bytes": dwl.n_seq * dwl.h_v * dwl.dk * dwl.dv * 4},
               "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
-                           "frac": dach / hbm, "traffic": None,
+                           "frac": dach / hbm,
+                           "traffic": recorded_traffic("decode_256seq_h32.md",
+                                                       "gated_delta_rule_160_b200/csrc/decode.cu"),
                            "peak_source": f"{peak_src} hbm_gbs",
                            "algorithmic_bytes_per_launch": dbytes}}
     del S, dec_in
