@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(HERE, "libgdn2.so")
 GDN2_F32, GDN2_BF16 = 0, 1
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_CUDA"}
 ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_decode_step",
-                 "gdn2_last_error_string", "gdn2_version")
+                 "gdn2_chunk_fwd_noalloc", "gdn2_last_error_string", "gdn2_version")
 
 
 class Gdn2Error(RuntimeError):
@@ -52,6 +52,8 @@ def load_library(path: str = LIB_PATH):
     lib.gdn2_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(Shape), ctypes.c_int]
     lib.gdn2_chunk_fwd.restype = ctypes.c_int
     lib.gdn2_chunk_fwd.argtypes = [ctypes.POINTER(Shape)] + [vp] * 10 + [vp, sz, vp]
+    lib.gdn2_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(Shape)] + [vp] * 10 + [vp]
     lib.gdn2_decode_step.restype = ctypes.c_int
     lib.gdn2_decode_step.argtypes = [ctypes.POINTER(Shape)] + [vp] * 9
     lib.gdn2_last_error_string.restype = ctypes.c_char_p
@@ -122,6 +124,23 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=Non
     _check(lib.gdn2_chunk_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                               _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
                               _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    return o, S_T
+
+
+def gdn2_chunk_fwd_noalloc(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
+                           o=None, S_T=None, stream=None):
+    """gdn2_chunk_fwd without a workspace, for callers that cannot allocate device memory:
+    the library keeps its packed-batch scratch in a static device array (at most 16384
+    sequences per call; calls that run concurrently on the GPU must not overlap). ``o`` and
+    ``S_T`` are required here -- this entry point allocates nothing."""
+    lib = load_library()
+    if o is None or S_T is None:
+        raise ValueError("gdn2_chunk_fwd_noalloc writes into caller-provided o and S_T")
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
+    shape = make_shape(q, v, n, o.dtype)
+    _check(lib.gdn2_chunk_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                      _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
+                                      _stream_handle(stream)))
     return o, S_T
 
 

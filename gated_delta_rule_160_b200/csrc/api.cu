@@ -93,6 +93,9 @@ Params make_params(const gdn2_shape* sh, const void* q, const void* k, const voi
 }
 
 }  // namespace
+
+gdn2_status report_error(gdn2_status st, const char* msg) { return fail(st, "%s", msg); }
+
 }  // namespace gdn2
 
 using namespace gdn2;

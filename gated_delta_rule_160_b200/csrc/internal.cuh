@@ -53,5 +53,7 @@ cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s)
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt);
 cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);
 cudaError_t read_tc_fault(unsigned int* out);
+// Record a failure in the calling thread's error string and return st.
+gdn2_status report_error(gdn2_status st, const char* msg);
 
 }  // namespace gdn2

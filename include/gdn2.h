@@ -117,6 +117,28 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_shape* shape,
                              const float* log_alpha, const void* b, const void* w,
                              float* S, void* o, gdn2_stream_t stream);
 
+/*
+ * Prefill for callers that cannot allocate device memory. The pages have no counterpart:
+ * this is an interface choice. It computes exactly what gdn2_chunk_fwd computes (same
+ * kernels, same arguments, no workspace), for callers that have no way to give the
+ * library scratch memory: code that owns no device allocator (a plug-in living inside
+ * another runtime's memory pool), code that must not allocate after start-up (a serving
+ * loop with a fixed memory budget), or code where a cudaMalloc would synchronise the
+ * device at the wrong moment. The scratch that packed batches need (the longest-first
+ * order of the sequences) lives in a 64 KB array inside the library image instead, held
+ * by every GPU that loads the library until the process exits.
+ * Limits: with cu_seqlens, at most 16384 sequences per call (more: GDN2_ERR_INVALID_ARG,
+ * nothing queued). All calls on a device share that array; each call writes every entry
+ * it reads, but calls whose work overlaps on the GPU (concurrent streams) race on it. The
+ * first call on each device looks the array up with that device current: make it before
+ * any stream capture. Nothing is allocated by this call.
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
+                                    const void* q, const void* k, const void* v,
+                                    const float* log_alpha, const void* b, const void* w,
+                                    const float* S0, const int32_t* cu_seqlens,
+                                    void* o, float* S_T, gdn2_stream_t stream);
+
 /* Description of the calling thread's last failure ("" if none). Never NULL. */
 GDN2_API const char* gdn2_last_error_string(void);
 
