@@ -26,15 +26,18 @@
 //
 // Phases per chunk (all 256 threads take part in each; thread t serves tensor-memory lane
 // t % 128 and column half t / 128):
-//   1 prep    load the chunk, cumsum log-decays, write the operand tiles
+//   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63)
 //   3 Gram epilogue + fp32 blocked triangular solve for T (16 -> 32 -> 64)
 //   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
 //   5 state epilogue: U <- f (.) U, Sref^T tile
 //   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term)
 //   7 Y tile  8 MMA R^T = Y^T T^T  9 -R tile  10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
-//   11 o epilogue (fp32 or bf16 stores)
-// The next chunk's rows are prefetched into L2 while the current one is processed.
+//   11 o epilogue (full fp32 chunks: one TMA store of a staged tile; else plain stores)
+// The next chunk's raw rows are staged by TMA while the current one is processed.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -55,12 +58,23 @@ constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exce
 constexpr uint32_t kTile = CH * D * 2;   // 16384
 constexpr uint32_t OFF_KH = 0;           // Kh      } rows 0..127 of the Gram B operand
 constexpr uint32_t OFF_QH = 1 * kTile;   // Qh hi   }
-constexpr uint32_t OFF_KBH = 2 * kTile;  // Kb hi   } rows 0..127 of the Gram A operand
-constexpr uint32_t OFF_E = 3 * kTile;    // Eb      }
-constexpr uint32_t OFF_KBL = 4 * kTile;  // Kb lo   (rows 64..127 of its operand are masked out)
-constexpr uint32_t OFF_XH = 5 * kTile;   // X hi
-constexpr uint32_t OFF_XL = 6 * kTile;   // X lo
-constexpr uint32_t OFF_QL = 7 * kTile;   // Qh lo
+constexpr uint32_t OFF_QL = 2 * kTile;   // Qh lo
+constexpr uint32_t OFF_KBH = 3 * kTile;  // Kb hi   } rows 0..127 of the Gram A operand
+constexpr uint32_t OFF_E = 4 * kTile;    // Eb      }
+constexpr uint32_t OFF_KBL = 5 * kTile;  // Kb lo   (rows 64..127 of its operand are masked out)
+constexpr uint32_t OFF_XH = 6 * kTile;   // X hi
+constexpr uint32_t OFF_XL = 7 * kTile;   // X lo
+// Raw chunk inputs, copied by TMA in boxes of 64 tokens x 128 bytes (64 bf16 or 32 fp32
+// channels) with the 128-byte swizzle: within each 8-row group the 16-byte chunk c of
+// row r sits at chunk c ^ (r % 8), so the prep's reads (8 rows, same columns) hit distinct
+// banks. A bf16 [64][128] tile is 2 boxes (8 KB each), an fp32 one 4 boxes. log_alpha and q
+// land where Kh / Qh / Ql live and v, w over Sref^T (both free once the state read of the
+// previous chunk is done); k, b land over Y^T / -R^T (free once the state MMAs are done).
+constexpr uint32_t OFF_RAW_LA = 0;           // fp32, 32 KB
+constexpr uint32_t OFF_RAW_Q = 2 * kTile;    // bf16, 16 KB
+// The o tile of a full chunk is staged as fp32 [64 tokens][128 channels] over Kb hi / Eb
+// (free once the state MMAs are done) and written by one TMA store.
+constexpr uint32_t OFF_OST = 3 * kTile;      // fp32, 32 KB
 // [64][64] bf16 tiles. MN-major B operands B[n=i][k=j] written by the Gram epilogue:
 //   (i/8)*1024 + (j/8)*128 + (j%8)*16 + (i%8)*2     (SBO = 1024, LBO = 128)
 constexpr uint32_t kSmall = CH * CH * 2;  // 8192
@@ -76,8 +90,14 @@ constexpr uint32_t OFF_WM = OFF_WT + 64 * 65 * 4;     // fp32 scratch [32][33]
 // Row-per-lane tiles [m][k] written by epilogues, K-major, K groups outermost:
 //   (k/8)*2048 + (m/8)*128 + (m%8)*16 + (k%8)*2     (LBO = 2048, SBO = 128)
 constexpr uint32_t OFF_SH = OFF_REG;              // Sref^T (bf16) [128][128]
-constexpr uint32_t OFF_Y = OFF_REG;               // Y^T [128][64]
-constexpr uint32_t OFF_R = OFF_REG + kTile;       // -R^T [128][64]
+constexpr uint32_t OFF_Y = OFF_REG + 2 * kTile;   // Y^T [128][64]
+constexpr uint32_t OFF_R = OFF_REG + 3 * kTile;   // -R^T [128][64]
+// raw v, w (bf16, 16 KB each) land over Sref^T once the state read is done; raw k, b over
+// Y^T / -R^T once the state MMAs are done
+constexpr uint32_t OFF_RAW_V = OFF_REG;
+constexpr uint32_t OFF_RAW_W = OFF_REG + kTile;
+constexpr uint32_t OFF_RAW_K = OFF_REG + 2 * kTile;
+constexpr uint32_t OFF_RAW_B = OFF_REG + 3 * kTile;
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128], f[128]
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 5 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
@@ -91,7 +111,14 @@ constexpr uint32_t TM_D1 = 128;  // [Y^T | O^T]
 constexpr uint32_t TM_R = 256;   // R^T
 constexpr uint32_t TM_U = 384;   // state, lanes m (value channel), cols c (key channel)
 
-enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45 };
+enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAW1, MB_RAW2, MB_RAW3 };
+
+// Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
+// 64 tokens with the 128-byte swizzle.
+struct RawMaps {
+    CUtensorMap la, q, k, b, v, w;
+    CUtensorMap o;  // fp32 output, used for full chunks (box {128, 1, 64}, no swizzle)
+};
 
 __device__ unsigned int g_tc_fault = 0;
 
@@ -102,12 +129,18 @@ __device__ __forceinline__ uint32_t off_lane_k(int m, int k) {     // epilogue t
     return (uint32_t)((k >> 3) * 2048 + (m >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2);
 }
 
+// Byte offsets of (token i, channel c) in the swizzled raw tiles (see the map above).
+__device__ __forceinline__ uint32_t raw_off_bf16(int i, int c) {
+    return (uint32_t)((c >> 6) * 8192 + i * 128 + ((((c & 63) >> 3) ^ (i & 7)) << 4) + (c & 7) * 2);
+}
+__device__ __forceinline__ uint32_t raw_off_f32(int i, int c) {
+    return (uint32_t)((c >> 5) * 8192 + i * 128 + ((((c & 31) >> 2) ^ (i & 7)) << 4) + (c & 3) * 4);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
-
 // Split 2 fp32 values into bf16 hi (packed) and bf16 lo = x - hi (packed): hi + lo carries
 // about 16 significant bits.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
@@ -136,7 +169,11 @@ __device__ __forceinline__ void store8_bf16(uint8_t* smem, uint32_t off, const f
 }
 
 template <typename TO>
-__global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
+constexpr bool kTmaStoreO = sizeof(TO) == 4;  // the o tensor map is fp32
+
+template <typename TO>
+__global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__ Params p,
+                                                          const __grid_constant__ RawMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = tid & 127;   // tensor-memory lane served by this thread
@@ -160,11 +197,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
     const int nchunks = (t1 - t0 + CH - 1) / CH;
     const size_t soff = ((size_t)n * p.h_v + h) * D * D;
 
-    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(p.q);
-    const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(p.k);
-    const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(p.v);
-    const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
-    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(p.w);
     TO* op = static_cast<TO*>(p.o);
 
     if (nchunks == 0) {  // empty sequence: S_T = S0
@@ -174,7 +206,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
     }
 
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(mbar(i), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(mbar(i), 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
@@ -188,6 +220,35 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
     const int tl = lane & 7;
     const int c0 = 16 * warp + 4 * (lane >> 3);
 
+    // raw inputs of a chunk, in three groups by when their space frees up:
+    // log_alpha, q, v, w (after the state read) and k, b (after the state MMAs)
+    auto issue_raw1 = [&](int ts) {
+        mbar_expect_tx(mbar(MB_RAW1), 3 * kTile);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+            tma_load_3d(sbase + OFF_RAW_LA + x * 8192, &maps.la, 32 * x, h, ts, mbar(MB_RAW1));
+#pragma unroll
+        for (int x = 0; x < 2; ++x) tma_load_3d(sbase + OFF_RAW_Q + x * 8192, &maps.q, 64 * x, g, ts, mbar(MB_RAW1));
+        mbar_expect_tx(mbar(MB_RAW2), 2 * kTile);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_load_3d(sbase + OFF_RAW_V + x * 8192, &maps.v, 64 * x, h, ts, mbar(MB_RAW2));
+            tma_load_3d(sbase + OFF_RAW_W + x * 8192, &maps.w, 64 * x, h, ts, mbar(MB_RAW2));
+        }
+    };
+    auto issue_raw3 = [&](int ts) {
+        mbar_expect_tx(mbar(MB_RAW3), 2 * kTile);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_load_3d(sbase + OFF_RAW_K + x * 8192, &maps.k, 64 * x, g, ts, mbar(MB_RAW3));
+            tma_load_3d(sbase + OFF_RAW_B + x * 8192, &maps.b, 64 * x, h, ts, mbar(MB_RAW3));
+        }
+    };
+    if (tid == 0) {
+        issue_raw1(t0);
+        issue_raw3(t0);
+    }
+
     for (int ci = 0; ci < nchunks; ++ci) {
         const int tc0 = t0 + ci * CH;
         const int nvalid = min(CH, t1 - tc0);
@@ -196,41 +257,44 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
 
         // ------------------------------------------------------------ 1. prep
         {
-            // every load of the chunk is issued before any arithmetic (8 passes x 6 loads in flight)
+            // the chunk's raw rows arrive by TMA; tokens past the sequence end read as zero
             float4 la[8];
             uint2 kq[8], qq[8], bq[8], vq[8], wq[8];
+            fault |= !mbar_wait(mbar(MB_RAW1), par, kWaitNs);
 #pragma unroll
             for (int pss = 0; pss < 8; ++pss) {
                 const int i = 8 * pss + tl;
                 const bool valid = i < nvalid;
-                const size_t tq = ((size_t)(tc0 + i) * p.h_qk + g) * D + c0;
-                const size_t tv = ((size_t)(tc0 + i) * p.h_v + h) * D + c0;
-                const uint2 z = make_uint2(0u, 0u);
-                la[pss] = valid ? *reinterpret_cast<const float4*>(p.log_alpha + tv) : make_float4(0.f, 0.f, 0.f, 0.f);
-                kq[pss] = valid ? *reinterpret_cast<const uint2*>(kp + tq) : z;
-                qq[pss] = valid ? *reinterpret_cast<const uint2*>(qp + tq) : z;
-                bq[pss] = valid ? *reinterpret_cast<const uint2*>(bp + tv) : z;
-                vq[pss] = valid ? *reinterpret_cast<const uint2*>(vp + tv) : z;
-                wq[pss] = valid ? *reinterpret_cast<const uint2*>(wp + tv) : z;
+                la[pss] = valid ? *reinterpret_cast<const float4*>(smem + OFF_RAW_LA + raw_off_f32(i, c0))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                qq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_Q + raw_off_bf16(i, c0))
+                                : make_uint2(0u, 0u);
             }
-            if (ci + 1 < nchunks) {
-                // bring the next chunk's rows into L2 (14 lines of 128 B per token) while
-                // this one is processed; one line per instruction keeps the issue cheap
-                const int tn = tc0 + CH;
-                const int nn = min(CH, t1 - tn);
-                for (int idx = tid; idx < nn * 14; idx += NT) {
-                    const int r = idx / 14, ln = idx % 14;
-                    const size_t tq = ((size_t)(tn + r) * p.h_qk + g) * D;
-                    const size_t tv = ((size_t)(tn + r) * p.h_v + h) * D;
-                    const char* a;
-                    if (ln < 2) a = reinterpret_cast<const char*>(qp + tq) + 128 * ln;
-                    else if (ln < 4) a = reinterpret_cast<const char*>(kp + tq) + 128 * (ln - 2);
-                    else if (ln < 6) a = reinterpret_cast<const char*>(vp + tv) + 128 * (ln - 4);
-                    else if (ln < 8) a = reinterpret_cast<const char*>(wp + tv) + 128 * (ln - 6);
-                    else if (ln < 10) a = reinterpret_cast<const char*>(bp + tv) + 128 * (ln - 8);
-                    else a = reinterpret_cast<const char*>(p.log_alpha + tv) + 128 * (ln - 10);
-                    prefetch_line_l2(a);
-                }
+            fault |= !mbar_wait(mbar(MB_RAW2), par, kWaitNs);
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                const bool valid = i < nvalid;
+                const uint32_t o = raw_off_bf16(i, c0);
+                const uint2 z = make_uint2(0u, 0u);
+                vq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_V + o) : z;
+                wq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_W + o) : z;
+            }
+            fault |= !mbar_wait(mbar(MB_RAW3), par, kWaitNs);
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                const bool valid = i < nvalid;
+                const uint32_t o = raw_off_bf16(i, c0);
+                const uint2 z = make_uint2(0u, 0u);
+                kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
+                bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
+            }
+            // the tiles written below overwrite the raw log_alpha / q rows and the staged o tile
+            if (tid == 0) bulk_wait_read0();
+            if (__syncthreads_or(fault)) {
+                fault = true;
+                break;
             }
             float G[8][4];
             float carry[4] = {0.f, 0.f, 0.f, 0.f};
@@ -529,6 +593,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
+        if (tid == 0 && ci + 1 < nchunks) issue_raw1(tc0 + CH);  // Kh / Qh / Ql and Sref^T are free now
 
         // ------------------------------------------------------------ 7. Y^T tile
         {
@@ -592,21 +657,37 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
         fault |= !mbar_wait(mbar(MB_45), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
+        if (tid == 0 && ci + 1 < nchunks) issue_raw3(tc0 + CH);  // Y^T / -R^T are dead now
 
         // ------------------------------------------------------------ 11. o
         {
             float ov[32];
             tmem_ld32(tmem + lane_bits + TM_D1 + 64 + 32 * hf, ov);
             tmem_wait_ld();
+            if (kTmaStoreO<TO> && nvalid == CH) {
+                // stage the fp32 tile [token][channel] and let one TMA store write it
+                float* ost = reinterpret_cast<float*>(smem + OFF_OST);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int i = 32 * hf + e;
-                if (i < nvalid) op[((size_t)(tc0 + i) * p.h_v + h) * D + L] = from_f32<TO>(ov[e]);
+                for (int e = 0; e < 32; ++e) ost[(32 * hf + e) * D + L] = ov[e];
+                fence_proxy_async_smem();
+                __syncthreads();
+                if (tid == 0) {
+                    tma_store_3d(&maps.o, sbase + OFF_OST, 0, h, tc0);
+                    bulk_commit();
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * hf + e;
+                    if (i < nvalid) op[((size_t)(tc0 + i) * p.h_v + h) * D + L] = from_f32<TO>(ov[e]);
+                }
             }
         }
         tc_fence_before();
         __syncthreads();
     }
+    // the staged o tile must be read out before shared memory is released or rewritten
+    if (tid == 0) bulk_wait_read0();
 
     if (!fault && p.S_T) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
@@ -630,20 +711,62 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(Params p) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;  // same value from every thread
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Rows of one head of a [T, heads, 128] tensor, in boxes of 64 tokens. swizzled: boxes of
+// 128 bytes per row (64 bf16 / 32 fp32 channels) with the 128-byte swizzle; else whole rows.
+bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap* m, const void* base, bool fp32, int heads,
+                 int T, bool swizzled) {
+    const cuuint64_t es = fp32 ? 4 : 2;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)heads * D * es};
+    cuuint32_t box[3] = {swizzled ? (cuuint32_t)(128 / es) : (cuuint32_t)D, 1u, (cuuint32_t)CH};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename TO>
 cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return cudaErrorNotSupported;
+    RawMaps maps;
+    if (!encode_rows(fn, &maps.la, p.log_alpha, true, p.h_v, p.T_total, true) ||
+        !encode_rows(fn, &maps.q, p.q, false, p.h_qk, p.T_total, true) ||
+        !encode_rows(fn, &maps.k, p.k, false, p.h_qk, p.T_total, true) ||
+        !encode_rows(fn, &maps.b, p.b, false, p.h_v, p.T_total, true) ||
+        !encode_rows(fn, &maps.v, p.v, false, p.h_v, p.T_total, true) ||
+        !encode_rows(fn, &maps.w, p.w, false, p.h_v, p.T_total, true))
+        return cudaErrorInvalidValue;
+    if (sizeof(TO) == 4) {
+        if (!encode_rows(fn, &maps.o, p.o, true, p.h_v, p.T_total, false)) return cudaErrorInvalidValue;
+    } else {
+        maps.o = maps.la;  // unused: bf16 outputs take plain stores
+    }
     // set on every launch: the attribute is per device and the call costs microseconds
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<TO><<<p.n_seq * p.h_v, NT, SMEM_BYTES, s>>>(p);
+    chunk_tc_kernel<TO><<<p.n_seq * p.h_v, NT, SMEM_BYTES, s>>>(p, maps);
     return cudaGetLastError();
 }
 
 }  // namespace
 
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt) {
-    return dt == GDN2_BF16 && p.dk == D && p.dv == D;
+    return dt == GDN2_BF16 && p.dk == D && p.dv == D && p.T_total > 0;
 }
 
 cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s) {
