@@ -25,14 +25,18 @@
 // (A, B, Qm, T, Y, R) stays in plain bf16.
 //
 // Phases per chunk (all 256 threads take part in each; thread t serves tensor-memory lane
-// t % 128 and column half t / 128):
+// t % 128 and column half t / 128). The MMAs of phases 4 and 6 are issued before the UT
+// solve and run while the solve's SIMT work proceeds:
 //   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63)
 //   3 Gram epilogue + fp32 blocked triangular solve for T (16 -> 32 -> 64)
 //   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
-//   5 state epilogue: U <- f (.) U, Sref^T tile
+//   5 state epilogue: U <- f (.) U, Sref^T (bf16) into tensor memory
 //   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term)
-//   7 Y tile  8 MMA R^T = Y^T T^T  9 -R tile  10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
+//   7 Y^T (bf16, tensor memory)  8 MMA R^T = Y^T T^T  9 -R^T (bf16, tensor memory)
+//   10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
+// Sref^T, Y^T and -R^T are A operands read from tensor memory; the others come from shared
+// memory.
 //   11 o epilogue (full fp32 chunks: one TMA store of a staged tile; else plain stores)
 // The next chunk's raw rows are staged by TMA while the current one is processed.
 #include <cuda.h>
@@ -67,11 +71,13 @@ constexpr uint32_t OFF_XL = 7 * kTile;   // X lo
 // Raw chunk inputs, copied by TMA in boxes of 64 tokens x 128 bytes (64 bf16 or 32 fp32
 // channels) with the 128-byte swizzle: within each 8-row group the 16-byte chunk c of
 // row r sits at chunk c ^ (r % 8), so the prep's reads (8 rows, same columns) hit distinct
-// banks. A bf16 [64][128] tile is 2 boxes (8 KB each), an fp32 one 4 boxes. log_alpha and q
-// land where Kh / Qh / Ql live and v, w over Sref^T (both free once the state read of the
-// previous chunk is done); k, b land over Y^T / -R^T (free once the state MMAs are done).
-constexpr uint32_t OFF_RAW_LA = 0;           // fp32, 32 KB
-constexpr uint32_t OFF_RAW_Q = 2 * kTile;    // bf16, 16 KB
+// banks. A bf16 [64][128] tile is 2 boxes (8 KB each), an fp32 one 4 boxes.
+//   group A: log_alpha, v, w -> the reused region, free once the previous chunk's
+//            X [B;P]^T MMAs are done;
+//   group B: q, k, b         -> over Kh / Qh / Ql, free once its state read is done.
+constexpr uint32_t OFF_RAW_Q = 0;            // bf16, 16 KB each
+constexpr uint32_t OFF_RAW_K = 1 * kTile;
+constexpr uint32_t OFF_RAW_B = 2 * kTile;
 // The o tile of a full chunk is staged as fp32 [64 tokens][128 channels] over Kb hi / Eb
 // (free once the state MMAs are done) and written by one TMA store.
 constexpr uint32_t OFF_OST = 3 * kTile;      // fp32, 32 KB
@@ -84,20 +90,13 @@ constexpr uint32_t OFF_REG = OFF_T + kSmall;  // 64 KB reused by phases 3 / 5-6 
 constexpr uint32_t OFF_B = OFF_REG;             // B   } [B; P hi] is one 128-row operand
 constexpr uint32_t OFF_PH = OFF_REG + kSmall;   // P hi}
 constexpr uint32_t OFF_PL = OFF_REG + 2 * kSmall;
-constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][65]
-constexpr uint32_t OFF_WT = OFF_WA + 64 * 65 * 4;     // fp32 T [64][65]
-constexpr uint32_t OFF_WM = OFF_WT + 64 * 65 * 4;     // fp32 scratch [32][33]
-// Row-per-lane tiles [m][k] written by epilogues, K-major, K groups outermost:
-//   (k/8)*2048 + (m/8)*128 + (m%8)*16 + (k%8)*2     (LBO = 2048, SBO = 128)
-constexpr uint32_t OFF_SH = OFF_REG;              // Sref^T (bf16) [128][128]
-constexpr uint32_t OFF_Y = OFF_REG + 2 * kTile;   // Y^T [128][64]
-constexpr uint32_t OFF_R = OFF_REG + 3 * kTile;   // -R^T [128][64]
-// raw v, w (bf16, 16 KB each) land over Sref^T once the state read is done; raw k, b over
-// Y^T / -R^T once the state MMAs are done
-constexpr uint32_t OFF_RAW_V = OFF_REG;
-constexpr uint32_t OFF_RAW_W = OFF_REG + kTile;
-constexpr uint32_t OFF_RAW_K = OFF_REG + 2 * kTile;
-constexpr uint32_t OFF_RAW_B = OFF_REG + 3 * kTile;
+constexpr int WS = 68;                                // fp32 row stride (16-byte aligned rows)
+constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][WS]
+constexpr uint32_t OFF_WT = OFF_WA + 64 * WS * 4;     // fp32 T [64][WS]
+constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
+constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
+constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
+constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128], f[128]
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 5 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
@@ -110,8 +109,11 @@ constexpr uint32_t TM_G = 0;     // Gram (transposed): lanes [Kb j ; Eb j], cols
 constexpr uint32_t TM_D1 = 128;  // [Y^T | O^T]
 constexpr uint32_t TM_R = 256;   // R^T
 constexpr uint32_t TM_U = 384;   // state, lanes m (value channel), cols c (key channel)
+constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 64 columns
+// Y^T and -R^T also serve as bf16 A operands from tensor memory, packed over the first 32
+// columns of their own fp32 accumulators (TM_D1, TM_R).
 
-enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAW1, MB_RAW2, MB_RAW3 };
+enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB };
 
 // Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
 // 64 tokens with the 128-byte swizzle.
@@ -124,9 +126,6 @@ __device__ unsigned int g_tc_fault = 0;
 
 __device__ __forceinline__ uint32_t off_rowmajor(int r, int c) {  // prep tiles, 128 channels
     return (uint32_t)((r >> 3) * 2048 + (c >> 3) * 128 + (r & 7) * 16 + (c & 7) * 2);
-}
-__device__ __forceinline__ uint32_t off_lane_k(int m, int k) {     // epilogue tiles, 128 lanes
-    return (uint32_t)((k >> 3) * 2048 + (m >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2);
 }
 
 // Byte offsets of (token i, channel c) in the swizzled raw tiles (see the map above).
@@ -206,7 +205,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     }
 
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(mbar(i), 1);
+        for (int i = 0; i < 7; ++i) mbar_init(mbar(i), 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
@@ -220,33 +219,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const int tl = lane & 7;
     const int c0 = 16 * warp + 4 * (lane >> 3);
 
-    // raw inputs of a chunk, in three groups by when their space frees up:
-    // log_alpha, q, v, w (after the state read) and k, b (after the state MMAs)
-    auto issue_raw1 = [&](int ts) {
-        mbar_expect_tx(mbar(MB_RAW1), 3 * kTile);
+    // raw inputs of a chunk in two groups, each issued as soon as its space frees up
+    auto issue_raw_a = [&](int ts) {  // log_alpha, v, w
+        mbar_expect_tx(mbar(MB_RAWA), 4 * kTile);
 #pragma unroll
         for (int x = 0; x < 4; ++x)
-            tma_load_3d(sbase + OFF_RAW_LA + x * 8192, &maps.la, 32 * x, h, ts, mbar(MB_RAW1));
-#pragma unroll
-        for (int x = 0; x < 2; ++x) tma_load_3d(sbase + OFF_RAW_Q + x * 8192, &maps.q, 64 * x, g, ts, mbar(MB_RAW1));
-        mbar_expect_tx(mbar(MB_RAW2), 2 * kTile);
+            tma_load_3d(sbase + OFF_RAW_LA + x * 8192, &maps.la, 32 * x, h, ts, mbar(MB_RAWA));
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            tma_load_3d(sbase + OFF_RAW_V + x * 8192, &maps.v, 64 * x, h, ts, mbar(MB_RAW2));
-            tma_load_3d(sbase + OFF_RAW_W + x * 8192, &maps.w, 64 * x, h, ts, mbar(MB_RAW2));
+            tma_load_3d(sbase + OFF_RAW_V + x * 8192, &maps.v, 64 * x, h, ts, mbar(MB_RAWA));
+            tma_load_3d(sbase + OFF_RAW_W + x * 8192, &maps.w, 64 * x, h, ts, mbar(MB_RAWA));
         }
     };
-    auto issue_raw3 = [&](int ts) {
-        mbar_expect_tx(mbar(MB_RAW3), 2 * kTile);
+    auto issue_raw_b = [&](int ts) {  // q, k, b
+        mbar_expect_tx(mbar(MB_RAWB), 3 * kTile);
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-            tma_load_3d(sbase + OFF_RAW_K + x * 8192, &maps.k, 64 * x, g, ts, mbar(MB_RAW3));
-            tma_load_3d(sbase + OFF_RAW_B + x * 8192, &maps.b, 64 * x, h, ts, mbar(MB_RAW3));
+            tma_load_3d(sbase + OFF_RAW_Q + x * 8192, &maps.q, 64 * x, g, ts, mbar(MB_RAWB));
+            tma_load_3d(sbase + OFF_RAW_K + x * 8192, &maps.k, 64 * x, g, ts, mbar(MB_RAWB));
+            tma_load_3d(sbase + OFF_RAW_B + x * 8192, &maps.b, 64 * x, h, ts, mbar(MB_RAWB));
         }
     };
     if (tid == 0) {
-        issue_raw1(t0);
-        issue_raw3(t0);
+        issue_raw_a(t0);
+        issue_raw_b(t0);
     }
 
     for (int ci = 0; ci < nchunks; ++ci) {
@@ -257,44 +253,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 1. prep
         {
-            // the chunk's raw rows arrive by TMA; tokens past the sequence end read as zero
+            // group A: log_alpha, v, w (tokens past the sequence end read as zero)
             float4 la[8];
-            uint2 kq[8], qq[8], bq[8], vq[8], wq[8];
-            fault |= !mbar_wait(mbar(MB_RAW1), par, kWaitNs);
+            uint2 vq[8], wq[8];
+            fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
 #pragma unroll
             for (int pss = 0; pss < 8; ++pss) {
                 const int i = 8 * pss + tl;
                 const bool valid = i < nvalid;
+                const uint32_t o = raw_off_bf16(i, c0);
+                const uint2 z = make_uint2(0u, 0u);
                 la[pss] = valid ? *reinterpret_cast<const float4*>(smem + OFF_RAW_LA + raw_off_f32(i, c0))
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-                qq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_Q + raw_off_bf16(i, c0))
-                                : make_uint2(0u, 0u);
-            }
-            fault |= !mbar_wait(mbar(MB_RAW2), par, kWaitNs);
-#pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
-                const bool valid = i < nvalid;
-                const uint32_t o = raw_off_bf16(i, c0);
-                const uint2 z = make_uint2(0u, 0u);
                 vq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_V + o) : z;
                 wq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_W + o) : z;
-            }
-            fault |= !mbar_wait(mbar(MB_RAW3), par, kWaitNs);
-#pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
-                const bool valid = i < nvalid;
-                const uint32_t o = raw_off_bf16(i, c0);
-                const uint2 z = make_uint2(0u, 0u);
-                kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
-                bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
-            }
-            // the tiles written below overwrite the raw log_alpha / q rows and the staged o tile
-            if (tid == 0) bulk_wait_read0();
-            if (__syncthreads_or(fault)) {
-                fault = true;
-                break;
             }
             float G[8][4];
             float carry[4] = {0.f, 0.f, 0.f, 0.f};
@@ -334,16 +306,46 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     scal[256 + buf * 128 + c] = glast[e];
                 }
             }
+            // X = w (.) v tiles (their space holds nothing raw)
 #pragma unroll
             for (int pss = 0; pss < 8; ++pss) {
                 const int i = 8 * pss + tl;
-                float kf[4], qf[4], bf[4], vf[4], wf[4];
-                unpack4_bf16(kq[pss], kf);
-                unpack4_bf16(qq[pss], qf);
-                unpack4_bf16(bq[pss], bf);
+                float vf[4], wf[4];
                 unpack4_bf16(vq[pss], vf);
                 unpack4_bf16(wq[pss], wf);
-                float kh[4], qv[4], kb[4], eb[4], xv[4];
+                uint2 xh, xl;
+                split2(wf[0] * vf[0], wf[1] * vf[1], xh.x, xl.x);
+                split2(wf[2] * vf[2], wf[3] * vf[3], xh.y, xl.y);
+                const uint32_t o = off_rowmajor(i, c0);
+                *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
+                *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
+            }
+            // group B: q, k, b; the tiles below overwrite these rows and the staged o tile
+            uint2 qq[8], kq[8], bq[8];
+            fault |= !mbar_wait(mbar(MB_RAWB), par, kWaitNs);
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                const bool valid = i < nvalid;
+                const uint32_t o = raw_off_bf16(i, c0);
+                const uint2 z = make_uint2(0u, 0u);
+                qq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_Q + o) : z;
+                kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
+                bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
+            }
+            if (tid == 0) bulk_wait_read0();
+            if (__syncthreads_or(fault)) {
+                fault = true;
+                break;
+            }
+#pragma unroll
+            for (int pss = 0; pss < 8; ++pss) {
+                const int i = 8 * pss + tl;
+                float qf[4], kf[4], bf[4];
+                unpack4_bf16(qq[pss], qf);
+                unpack4_bf16(kq[pss], kf);
+                unpack4_bf16(bq[pss], bf);
+                float kh[4], qv[4], kb[4], eb[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float ge = exp2f(G[pss][e] - gref[e]);
@@ -352,15 +354,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     qv[e] = qf[e] * ge;
                     kb[e] = kf[e] * gi;
                     eb[e] = bf[e] * kf[e] * gi;
-                    xv[e] = wf[e] * vf[e];
                 }
-                uint2 qh, ql, kbh, kbl, xh, xl;
+                uint2 qh, ql, kbh, kbl;
                 split2(qv[0], qv[1], qh.x, ql.x);
                 split2(qv[2], qv[3], qh.y, ql.y);
                 split2(kb[0], kb[1], kbh.x, kbl.x);
                 split2(kb[2], kb[3], kbh.y, kbl.y);
-                split2(xv[0], xv[1], xh.x, xl.x);
-                split2(xv[2], xv[3], xh.y, xl.y);
                 const uint32_t o = off_rowmajor(i, c0);
                 store4_bf16(smem, OFF_KH + o, kh);
                 store4_bf16(smem, OFF_E + o, eb);
@@ -368,12 +367,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 *reinterpret_cast<uint2*>(smem + OFF_QL + o) = ql;
                 *reinterpret_cast<uint2*>(smem + OFF_KBH + o) = kbh;
                 *reinterpret_cast<uint2*>(smem + OFF_KBL + o) = kbl;
-                *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
-                *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
             }
         }
         fence_proxy_async_smem();
-        __syncthreads();
+        if (__syncthreads_or(fault)) { fault = true; break; }
 
         // ------------------------------------------------------------ 2. Gram MMAs
         if (tid == 0) {
@@ -434,7 +431,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
             } else if (hf == 0) {  // A_ij, j < i, fp32 for the solve
 #pragma unroll
-                for (int i = 0; i < 64; ++i) WA[i * 65 + j] = (i > j) ? val(i) : 0.f;
+                for (int i = 0; i < 64; ++i) WA[i * WS + j] = (i > j) ? val(i) : 0.f;
             } else {  // Qm_ij, j <= i
 #pragma unroll
                 for (int q8 = 0; q8 < 8; ++q8) {
@@ -444,86 +441,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     store8_bf16(smem, OFF_QM + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
                 }
             }
-        }
-        __syncthreads();
-        // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
-        // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
-        // and of 32 into 64 with T_21 = -T_22 (A_21 T_11).
-        if (tid < 64) {
-            const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
-            float x[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float s = 0.f;
-#pragma unroll
-                for (int l = 0; l < r; ++l) s += (l >= jj) ? WA[(16 * bI + r) * 65 + 16 * bI + l] * x[l] : 0.f;
-                x[r] = (r < jj) ? 0.f : (r == jj ? 1.f : -s);
-                WT[(16 * bI + r) * 65 + col] = x[r];
-            }
-        } else {
-            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
-                const int r = idx >> 6, c = idx & 63;
-                if ((c >> 4) > (r >> 4)) WT[r * 65 + c] = 0.f;
-            }
-        }
-        __syncthreads();
-        {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
-            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
-            float m0 = 0.f, m1 = 0.f;
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-                const float t = WT[(base + l) * 65 + base + c];
-                m0 += WA[(base + 16 + r0) * 65 + base + l] * t;
-                m1 += WA[(base + 24 + r0) * 65 + base + l] * t;
-            }
-            WM[((tid >> 7) * 16 + r0) * 33 + c] = m0;
-            WM[((tid >> 7) * 16 + r0 + 8) * 33 + c] = m1;
-        }
-        __syncthreads();
-        {   // level 2, step 2: T_10 = -T_11 M
-            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
-            const float* Mb = WM + (tid >> 7) * 16 * 33;
-            float t0 = 0.f, t1 = 0.f;
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-                const float mv = Mb[l * 33 + c];
-                if (l <= r0) t0 += WT[(base + 16 + r0) * 65 + base + 16 + l] * mv;
-                if (l <= r0 + 8) t1 += WT[(base + 24 + r0) * 65 + base + 16 + l] * mv;
-            }
-            WT[(base + 16 + r0) * 65 + base + c] = -t0;
-            WT[(base + 24 + r0) * 65 + base + c] = -t1;
-        }
-        __syncthreads();
-        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
-            const int c = tid & 31, r0 = tid >> 5;
-            float m[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int l = 0; l < 32; ++l) {
-                const float t = WT[l * 65 + c];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m[k] += WA[(32 + r0 + 8 * k) * 65 + l] * t;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) WM[(r0 + 8 * k) * 33 + c] = m[k];
-        }
-        __syncthreads();
-        {   // level 3, step 2: T_BA = -T_BB M
-            const int c = tid & 31, r0 = tid >> 5;
-            float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int l = 0; l < 32; ++l) {
-                const float mv = WM[l * 33 + c];
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (l <= r0 + 8 * k) t[k] += WT[(32 + r0 + 8 * k) * 65 + 32 + l] * mv;
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) WT[(32 + r0 + 8 * k) * 65 + c] = -t[k];
-        }
-        __syncthreads();
-        for (int idx = tid; idx < 512; idx += NT) {  // T as a K-major bf16 B operand [i][j]
-            const int i = idx & 63, jg = idx >> 6;
-            store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * 65 + 8 * jg]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -544,12 +461,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
             mma_commit(mbar(MB_2B));
         }
-        fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
-        if (__syncthreads_or(fault)) { fault = true; break; }
-        tc_fence_after();
-
         // ------------------------------------------------------------ 5. state epilogue
         {
+            uint32_t packed[32];
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
                 const int cb = 64 * hf + 32 * part;
@@ -568,11 +482,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
                 tmem_st32(tmem + lane_bits + TM_U + cb, u);
 #pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_SH + off_lane_k(L, cb + 8 * e8), &u[8 * e8]);
+                for (int e = 0; e < 16; ++e) packed[16 * part + e] = pack_bf16(u[2 * e], u[2 * e + 1]);
             }
+            // Sref^T as a bf16 A operand: key channels 64*hf .. +63 in columns 32*hf .. +31
+            float pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = __uint_as_float(packed[e]);
+            tmem_st32(tmem + lane_bits + TM_S + 32 * hf, pk);
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
@@ -583,27 +501,152 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_SH + ks * 4096, 2048, 128),
-                         sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
-                mma_bf16(tmem + TM_D1 + 64, sdesc(sbase + OFF_SH + ks * 4096, 2048, 128),
-                         sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
+                const uint32_t a = tmem + TM_S + ks * 8;
+                mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
+                mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
             }
             mma_commit(mbar(MB_2A));
         }
+        // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
+        // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
+        // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
+        // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
+        // (the same row for a whole warp: broadcast), columns as consecutive floats.
+        if (tid < 64) {
+            const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float* arow = WA + (16 * bI + r) * WS + 16 * bI;
+                float s = 0.f;
+#pragma unroll
+                for (int l4 = 0; l4 < 16; l4 += 4) {
+                    if (l4 < r) {
+                        const float4 a = *reinterpret_cast<const float4*>(arow + l4);
+                        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (l4 + u < r) s += (l4 + u >= jj) ? av[u] * x[l4 + u] : 0.f;
+                    }
+                }
+                x[r] = (r < jj) ? 0.f : (r == jj ? 1.f : -s);
+                WT[(16 * bI + r) * WS + col] = x[r];
+            }
+        } else {
+            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
+                const int r = idx >> 6, c = idx & 63;
+                if ((c >> 4) > (r >> 4)) WT[r * WS + c] = 0.f;
+            }
+        }
+        __syncthreads();
+        {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
+            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
+            const float* a0 = WA + (base + 16 + r0) * WS + base;
+            const float* a1 = WA + (base + 24 + r0) * WS + base;
+            float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+            for (int l4 = 0; l4 < 16; l4 += 4) {
+                const float4 x0 = *reinterpret_cast<const float4*>(a0 + l4);
+                const float4 x1 = *reinterpret_cast<const float4*>(a1 + l4);
+                const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float t = WT[(base + l4 + u) * WS + base + c];
+                    m0 += xa[u] * t;
+                    m1 += xb[u] * t;
+                }
+            }
+            WM[((tid >> 7) * 16 + r0) * 33 + c] = m0;
+            WM[((tid >> 7) * 16 + r0 + 8) * 33 + c] = m1;
+        }
+        __syncthreads();
+        {   // level 2, step 2: T_10 = -T_11 M
+            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
+            const float* Mb = WM + (tid >> 7) * 16 * 33;
+            const float* t0r = WT + (base + 16 + r0) * WS + base + 16;
+            const float* t1r = WT + (base + 24 + r0) * WS + base + 16;
+            float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+            for (int l4 = 0; l4 < 16; l4 += 4) {
+                const float4 y0 = *reinterpret_cast<const float4*>(t0r + l4);
+                const float4 y1 = *reinterpret_cast<const float4*>(t1r + l4);
+                const float ya[4] = {y0.x, y0.y, y0.z, y0.w}, yb[4] = {y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float mv = Mb[(l4 + u) * 33 + c];
+                    t0 += ya[u] * mv;  // T_11's upper triangle is stored as zeros
+                    t1 += yb[u] * mv;
+                }
+            }
+            WT[(base + 16 + r0) * WS + base + c] = -t0;
+            WT[(base + 24 + r0) * WS + base + c] = -t1;
+        }
+        __syncthreads();
+        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
+            const int c = tid & 31, r0 = tid >> 5;
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int l4 = 0; l4 < 32; l4 += 4) {
+                float tv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) tv[u] = WT[(l4 + u) * WS + c];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WA + (32 + r0 + 8 * k) * WS + l4);
+                    m[k] += a.x * tv[0] + a.y * tv[1] + a.z * tv[2] + a.w * tv[3];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) WM[(r0 + 8 * k) * 33 + c] = m[k];
+        }
+        __syncthreads();
+        {   // level 3, step 2: T_BA = -T_BB M (T_BB lower triangular, its upper part is zero)
+            const int c = tid & 31, r0 = tid >> 5;
+            float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int l4 = 0; l4 < 32; l4 += 4) {
+                float mv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mv[u] = WM[(l4 + u) * 33 + c];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WT + (32 + r0 + 8 * k) * WS + 32 + l4);
+                    t[k] += a.x * mv[0] + a.y * mv[1] + a.z * mv[2] + a.w * mv[3];
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) WT[(32 + r0 + 8 * k) * WS + c] = -t[k];
+        }
+        __syncthreads();
+        for (int idx = tid; idx < 512; idx += NT) {  // T as a K-major bf16 B operand [i][j]
+            const int i = idx & 63, jg = idx >> 6;
+            store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
-        if (tid == 0 && ci + 1 < nchunks) issue_raw1(tc0 + CH);  // Kh / Qh / Ql and Sref^T are free now
+        if (tid == 0 && ci + 1 < nchunks) {
+            issue_raw_a(tc0 + CH);  // B / P and the solve's workspace are dead
+            issue_raw_b(tc0 + CH);  // Kh / Qh / Ql are dead
+        }
 
-        // ------------------------------------------------------------ 7. Y^T tile
+        // ------------------------------------------------------------ 7. Y^T as a bf16 A operand
         {
             float y[32];
             tmem_ld32(tmem + lane_bits + TM_D1 + 32 * hf, y);
             tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-            for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_Y + off_lane_k(L, 32 * hf + 8 * e8), &y[8 * e8]);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(y[2 * e], y[2 * e + 1]);
+            __syncthreads();  // every half has read its fp32 columns before any are overwritten
+            tmem_st16(tmem + lane_bits + TM_D1 + 16 * hf, pk);
+            tmem_wait_st();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
@@ -613,25 +656,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int ks = 0; ks < CH / 16; ++ks)
-                mma_bf16(tmem + TM_R, sdesc(sbase + OFF_Y + ks * 4096, 2048, 128),
-                         sdesc(sbase + OFF_T + ks * 2048, 1024, 128), id64, ks > 0);
+                mma_bf16_ts(tmem + TM_R, tmem + TM_D1 + ks * 8, sdesc(sbase + OFF_T + ks * 2048, 1024, 128), id64,
+                            ks > 0);
             mma_commit(mbar(MB_3));
         }
         fault |= !mbar_wait(mbar(MB_3), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
 
-        // ------------------------------------------------------------ 9. -R^T tile
+        // ------------------------------------------------------------ 9. -R^T as a bf16 A operand
         {
             float r[32];
             tmem_ld32(tmem + lane_bits + TM_R + 32 * hf, r);
             tmem_wait_ld();
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = -r[e];
-#pragma unroll
-            for (int e8 = 0; e8 < 4; ++e8) store8_bf16(smem, OFF_R + off_lane_k(L, 32 * hf + 8 * e8), &r[8 * e8]);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(-r[2 * e], -r[2 * e + 1]);
+            __syncthreads();  // every half has read its fp32 columns before any are overwritten
+            tmem_st16(tmem + lane_bits + TM_R + 16 * hf, pk);
+            tmem_wait_st();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
@@ -643,21 +687,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const uint32_t id_rx = idesc_bf16(128, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < CH / 16; ++ks) {
-                const uint64_t rr = sdesc(sbase + OFF_R + ks * 4096, 2048, 128);
+                const uint32_t rr = tmem + TM_R + ks * 8;
                 const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
                 const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
-                mma_bf16(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
+                mma_bf16_ts(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
                 mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
                 mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
                 mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
-                mma_bf16(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
+                mma_bf16_ts(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
             }
             mma_commit(mbar(MB_45));
         }
         fault |= !mbar_wait(mbar(MB_45), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
-        if (tid == 0 && ci + 1 < nchunks) issue_raw3(tc0 + CH);  // Y^T / -R^T are dead now
 
         // ------------------------------------------------------------ 11. o
         {
