@@ -53,7 +53,6 @@ using namespace tc;
 constexpr int CH = 64;   // chunk length
 constexpr int D = 128;   // dk = dv
 constexpr int NT = 256;  // threads per CTA
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
@@ -97,7 +96,7 @@ constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
 constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
 constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
-constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float g2ref[2][128], g2last[2][128], f[128]
+constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float gref[2][128], glast[2][128], f[128]
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 5 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
@@ -113,7 +112,7 @@ constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 6
 // Y^T and -R^T also serve as bf16 A operands from tensor memory, packed over the first 32
 // columns of their own fp32 accumulators (TM_D1, TM_R).
 
-enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB };
+enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX };
 
 // Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
 // 64 tokens with the 128-byte swizzle.
@@ -179,7 +178,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const int hf = tid >> 7;   // column half
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
-    float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] g2ref, [256..511] g2last
+    float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast
     float* fscal = scal + 512;                                  // [128] state frame factors
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
     float* WT = reinterpret_cast<float*>(smem + OFF_WT);
@@ -205,7 +204,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     }
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(mbar(i), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(mbar(i), 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
@@ -272,7 +271,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             float carry[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int pss = 0; pss < 8; ++pss) {
-                float x[4] = {la[pss].x * kLog2e, la[pss].y * kLog2e, la[pss].z * kLog2e, la[pss].w * kLog2e};
+                float x[4] = {la[pss].x, la[pss].y, la[pss].z, la[pss].w};
 #pragma unroll
                 for (int dlt = 1; dlt < 8; dlt <<= 1) {
 #pragma unroll
@@ -300,8 +299,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     const int c = c0 + e;
                     // factor taking the state from the previous chunk's reference frame (or
                     // S0) into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
-                    fscal[c] = ci == 0 ? exp2f(gref[e])
-                                       : exp2f(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref[e]);
+                    fscal[c] = ci == 0 ? expf(gref[e])
+                                       : expf(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref[e]);
                     scal[buf * 128 + c] = gref[e];
                     scal[256 + buf * 128 + c] = glast[e];
                 }
@@ -348,8 +347,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 float kh[4], qv[4], kb[4], eb[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float ge = exp2f(G[pss][e] - gref[e]);
-                    const float gi = exp2f(gref[e] - G[pss][e]);
+                    // fast exponential: relative error a few 1e-6 for |arguments| up to ~45,
+                    // well below the 2^-16 carried by the hi/lo operand splits
+                    const float ge = __expf(G[pss][e] - gref[e]);
+                    const float gi = __expf(gref[e] - G[pss][e]);
                     kh[e] = kf[e] * ge;
                     qv[e] = qf[e] * ge;
                     kb[e] = kf[e] * gi;
@@ -383,6 +384,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 mma_bf16(tmem + TM_G, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
                          sdesc(sbase + OFF_KH + kofs, 128, 2048), id128, ks > 0);
             }
+            mma_commit(mbar(MB_G));
             // P cross terms (lanes 0..63 hold Kb rows; lanes 64..127 are masked out)
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
                          sdesc(sbase + OFF_QL + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
             }
-            mma_commit(mbar(MB_G));
+            mma_commit(mbar(MB_GX));
         }
         fault |= !mbar_wait(mbar(MB_G), par, kWaitNs);
         if (__syncthreads_or(fault)) { fault = true; break; }
@@ -400,6 +402,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 3. Gram epilogue
         {
+            // warps 4..7 on lanes 0..63 read the P block, which the cross terms still update
+            if (hf == 1 && L < 64) {
+                if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
+                tc_fence_after();
+            }
             float v0[32], v1[32];
             tmem_ld32(tmem + lane_bits + TM_G + 64 * hf, v0);
             tmem_ld32(tmem + lane_bits + TM_G + 64 * hf + 32, v1);
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     for (int e = 0; e < 8; ++e) f[e] = (8 * q8 + e > j) ? val(8 * q8 + e) : 0.f;
                     store8_bf16(smem, OFF_B + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
                 }
-            } else if (L < 64) {  // P_ij, j <= i, split hi / lo
+            } else if (L < 64) {  // P_ij, j <= i, split hi / lo (after the cross terms)
 #pragma unroll
                 for (int q8 = 0; q8 < 8; ++q8) {
                     float x[8];
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(fault)) { fault = true; break; }
 
         // ------------------------------------------------------------ 4. D1 = X^T [B;P]^T
         if (tid == 0) {
@@ -508,6 +515,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             mma_commit(mbar(MB_2A));
         }
         // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
+        // The next chunk's q, k, b may land over Kh / Qh / Ql as soon as the Sref MMAs are
+        // done; thread 0 checks between the solve's levels and issues them then.
+        bool raw_b_issued = !(ci + 1 < nchunks);
+        auto try_issue_raw_b = [&]() {
+            if (tid == 0 && !raw_b_issued && mbar_test(mbar(MB_2A), par)) {
+                tc_fence_after();
+                issue_raw_b(tc0 + CH);
+                raw_b_issued = true;
+            }
+        };
         // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
         // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
         // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
@@ -539,6 +556,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         __syncthreads();
+        try_issue_raw_b();
         {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
             const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
             const float* a0 = WA + (base + 16 + r0) * WS + base;
@@ -582,6 +600,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             WT[(base + 24 + r0) * WS + base + c] = -t1;
         }
         __syncthreads();
+        try_issue_raw_b();
         {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
             const int c = tid & 31, r0 = tid >> 5;
             float m[4] = {0.f, 0.f, 0.f, 0.f};
@@ -631,8 +650,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         if (__syncthreads_or(fault)) { fault = true; break; }
         tc_fence_after();
         if (tid == 0 && ci + 1 < nchunks) {
-            issue_raw_a(tc0 + CH);  // B / P and the solve's workspace are dead
-            issue_raw_b(tc0 + CH);  // Kh / Qh / Ql are dead
+            issue_raw_a(tc0 + CH);                   // B / P and the solve's workspace are dead
+            if (!raw_b_issued) issue_raw_b(tc0 + CH);  // Kh / Qh / Ql are dead
         }
 
         // ------------------------------------------------------------ 7. Y^T as a bf16 A operand
@@ -744,7 +763,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
                 const int c = cb + e;
-                p.S_T[soff + (size_t)c * D + L] = u[e] * exp2f(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
+                p.S_T[soff + (size_t)c * D + L] = u[e] * expf(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
             }
         }
     }
