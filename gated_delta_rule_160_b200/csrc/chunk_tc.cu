@@ -1,6 +1,6 @@
 // chunk_tc.cu -- chunkwise-parallel prefill on the tcgen05 tensor cores (bf16 inputs,
-// dk = dv = 128, chunks of C = 64 tokens). One CTA of 256 threads owns one (sequence,
-// value head) and walks its chunks in order; the fp32 state lives in tensor memory.
+// dk = dv = 128, chunks of C = 64 tokens). One CTA owns one (sequence, value head) and
+// walks its chunks in order; the fp32 state lives in tensor memory.
 //
 // Chunk algebra (per chunk, state S on entry; e = b(.)k, x = w(.)v, G = inclusive cumsum
 // of log_alpha over the chunk, per key channel). Every decayed operand is taken relative
@@ -24,17 +24,19 @@
 // significant bits); Qh Sref splits Qh only (Qh_hi Sref + Qh_lo Sref); the erase path
 // (A, B, Qm, T, Y, R) stays in plain bf16.
 //
-// Phases per chunk (all 256 threads take part in each; thread t serves tensor-memory lane
-// t % 128 and column half t / 128). The MMAs of phases 4 and 6 are issued before the UT
-// solve and run while the solve's SIMT work proceeds:
+// Phases per chunk. Eight SIMT warps take part in each (thread t serves tensor-memory lane
+// t % 128 and column half t / 128); a ninth warp only issues the MMA groups, each as soon
+// as the SIMT warps signal that its operands are written, so no SIMT warp waits behind the
+// tensor pipe. The MMAs of phases 4 and 6 run while the UT solve's SIMT work proceeds:
 //   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
-//   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63)
+//   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
+//             written while they run
 //   3 Gram epilogue + fp32 blocked triangular solve for T (16 -> 32 -> 64)
 //   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
 //   5 state epilogue: U <- f (.) U, Sref^T (bf16) into tensor memory
-//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term)
+//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term), then U += X^T Kb (no state read)
 //   7 Y^T (bf16, tensor memory)  8 MMA R^T = Y^T T^T  9 -R^T (bf16, tensor memory)
-//   10 MMA: O^T -= R^T Qm^T, U += X^T Kb - R^T Eb
+//   10 MMA: O^T -= R^T Qm^T, U -= R^T Eb
 // Sref^T, Y^T and -R^T are A operands read from tensor memory; the others come from shared
 // memory.
 //   11 o epilogue (full fp32 chunks: one TMA store of a staged tile; else plain stores)
@@ -52,7 +54,9 @@ using namespace tc;
 
 constexpr int CH = 64;   // chunk length
 constexpr int D = 128;   // dk = dv
-constexpr int NT = 256;  // threads per CTA
+constexpr int NS = 256;           // SIMT threads (warps 0..7): prep, epilogues, solve
+constexpr int kIssuer = NS / 32;  // warp 8 issues every MMA
+constexpr int NT = NS + 32;       // threads per CTA
 constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
@@ -96,9 +100,10 @@ constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
 constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
 constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
-constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;  // float gref[2][128], glast[2][128], f[128]
-constexpr uint32_t OFF_MBAR = OFF_SCAL + 5 * 128 * 4;
-constexpr uint32_t OFF_TSLOT = OFF_MBAR + 8 * 8;
+// float gref[2][128], glast[2][128], f[128], half-chunk log-decay totals [2][128]
+constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
+constexpr uint32_t OFF_MBAR = OFF_SCAL + 7 * 128 * 4;
+constexpr uint32_t OFF_TSLOT = OFF_MBAR + 16 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
 static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -112,7 +117,10 @@ constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 6
 // Y^T and -R^T also serve as bf16 A operands from tensor memory, packed over the first 32
 // columns of their own fp32 accumulators (TM_D1, TM_R).
 
-enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX };
+// MB_*: MMA groups done (committed by the issuer warp) and raw rows landed (TMA);
+// RDY_*: operands of an MMA group written (one arrival from the SIMT warps).
+enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX, RDY_G, RDY_2B, RDY_2A, RDY_3, RDY_45, kNumMbar };
+static_assert(kNumMbar <= 16, "mbarrier slots");
 
 // Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
 // 64 tokens with the 128-byte swizzle.
@@ -180,6 +188,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
     float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast
     float* fscal = scal + 512;                                  // [128] state frame factors
+    float* htot = scal + 640;  // [2][128] sums of log_alpha over tokens 0..31 and 32..63
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
     float* WT = reinterpret_cast<float*>(smem + OFF_WT);
     float* WM = reinterpret_cast<float*>(smem + OFF_WM);
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     }
 
     if (tid == 0) {
-        for (int i = 0; i < 8; ++i) mbar_init(mbar(i), 1);
+        for (int i = 0; i < kNumMbar; ++i) mbar_init(mbar(i), 1);
         fence_mbar_init();
     }
     if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
@@ -244,7 +253,108 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         issue_raw_b(t0);
     }
 
-    for (int ci = 0; ci < nchunks; ++ci) {
+    if (warp == kIssuer) {
+        // One thread of the issuer warp waits for each MMA group's operands, issues the group
+        // and commits it to the group's completion barrier, chunk after chunk, so that no
+        // SIMT warp stalls behind the tensor pipe. If the SIMT warps stop early (a fault), the
+        // next wait here runs out and this warp stops too.
+        if (lane == 0) {
+            const uint32_t sbase_k = sbase, tmem_k = tmem;
+            for (int ci = 0; ci < nchunks; ++ci) {
+                const uint32_t par = (uint32_t)(ci & 1);
+                // addresses re-derived every chunk: kept live across the loop, the ~80 operand
+                // descriptors would take the registers the SIMT warps need
+                const uint32_t sbase = opaque_u32(sbase_k), tmem = opaque_u32(tmem_k);
+                if (!mbar_wait(mbar(RDY_G), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // Gram: [Kb; Eb] x [Kh; Qh]^T, then the P cross terms
+                    const uint32_t id128 = idesc_bf16(128, 128, false, false);
+                    const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t kofs = ks * 256;
+                        mma_bf16(tmem + TM_G, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
+                                 sdesc(sbase + OFF_KH + kofs, 128, 2048), id128, ks > 0);
+                    }
+                    mma_commit(mbar(MB_G));
+                    // P cross terms (lanes 0..63 hold Kb rows; lanes 64..127 are masked out)
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t kofs = ks * 256;
+                        mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBL + kofs, 128, 2048),
+                                 sdesc(sbase + OFF_QH + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
+                        mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
+                                 sdesc(sbase + OFF_QL + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
+                    }
+                    mma_commit(mbar(MB_GX));
+                }
+                if (!mbar_wait(mbar(RDY_2B), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // D1 = X^T [B; P]^T
+                    const uint32_t id128 = idesc_bf16(128, 128, true, true);
+                    const uint32_t id64 = idesc_bf16(128, 64, true, true);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks) {
+                        const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
+                        const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
+                        mma_bf16(tmem + TM_D1, xh, sdesc(sbase + OFF_B + ks * 256, 128, 1024), id128, ks > 0);
+                        mma_bf16(tmem + TM_D1 + 64, xl, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
+                        mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PL + ks * 256, 128, 1024), id64, 1u);
+                    }
+                    mma_commit(mbar(MB_2B));
+                }
+                if (!mbar_wait(mbar(RDY_2A), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // D1 += Sref^T [Kh; Qh]^T; then U += X^T Kb, which needs no state read
+                    const uint32_t id128 = idesc_bf16(128, 128, false, false);
+                    const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint32_t a = tmem + TM_S + ks * 8;
+                        mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
+                        mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
+                    }
+                    mma_commit(mbar(MB_2A));
+                    const uint32_t id_xx = idesc_bf16(128, 128, true, true);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks) {
+                        const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
+                        const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
+                        mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
+                        mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
+                        mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
+                    }
+                }
+                if (!mbar_wait(mbar(RDY_3), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // R^T = Y^T T^T
+                    const uint32_t id64 = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks)
+                        mma_bf16_ts(tmem + TM_R, tmem + TM_D1 + ks * 8, sdesc(sbase + OFF_T + ks * 2048, 1024, 128),
+                                    id64, ks > 0);
+                    mma_commit(mbar(MB_3));
+                }
+                if (!mbar_wait(mbar(RDY_45), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // O^T -= R^T Qm^T;  U -= R^T Eb
+                    const uint32_t id_o = idesc_bf16(128, 64, false, true);
+                    const uint32_t id_rx = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks) {
+                        const uint32_t rr = tmem + TM_R + ks * 8;
+                        mma_bf16_ts(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
+                        mma_bf16_ts(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
+                    }
+                    mma_commit(mbar(MB_45));
+                }
+            }
+        }
+        __syncwarp();
+    }
+    const int simt_chunks = warp == kIssuer ? 0 : nchunks;
+
+    for (int ci = 0; ci < simt_chunks; ++ci) {
         const int tc0 = t0 + ci * CH;
         const int nvalid = min(CH, t1 - tc0);
         const int buf = ci & 1;
@@ -252,72 +362,34 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 1. prep
         {
-            // group A: log_alpha, v, w (tokens past the sequence end read as zero)
-            float4 la[8];
-            uint2 vq[8], wq[8];
+            // group A: log_alpha, v, w (tokens past the sequence end count as zero); v and w
+            // are read after the Gram MMAs are under way.
+            // Cumulative log-decay G, in place over the staged log_alpha rows: thread
+            // (channel c, half hh) sums tokens 32hh .. 32hh + 31 of channel c. The upper half
+            // still lacks the lower half's total, which is added where G is read.
             fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
+            {
+                const int c = tid & 127, hh = tid >> 7;
+                float acc = 0.f;
 #pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
-                const bool valid = i < nvalid;
-                const uint32_t o = raw_off_bf16(i, c0);
-                const uint2 z = make_uint2(0u, 0u);
-                la[pss] = valid ? *reinterpret_cast<const float4*>(smem + OFF_RAW_LA + raw_off_f32(i, c0))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                vq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_V + o) : z;
-                wq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_W + o) : z;
-            }
-            float G[8][4];
-            float carry[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                float x[4] = {la[pss].x, la[pss].y, la[pss].z, la[pss].w};
-#pragma unroll
-                for (int dlt = 1; dlt < 8; dlt <<= 1) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float y = __shfl_up_sync(0xffffffffu, x[e], dlt, 8);
-                        if (tl >= dlt) x[e] += y;
-                    }
+                for (int r = 0; r < 32; ++r) {
+                    const int i = 32 * hh + r;
+                    float* gp = reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c));
+                    acc += i < nvalid ? *gp : 0.f;
+                    *gp = acc;
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    G[pss][e] = x[e] + carry[e];
-                    carry[e] = __shfl_sync(0xffffffffu, G[pss][e], (lane & 24) | 7);
-                }
+                htot[128 * hh + c] = acc;
             }
-            float gref[4], glast[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float gfirst = __shfl_sync(0xffffffffu, G[0][e], lane & 24);
-                glast[e] = carry[e];
-                gref[e] = 0.5f * (gfirst + glast[e]);
-            }
-            if (tl == 0) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int c = c0 + e;
-                    // factor taking the state from the previous chunk's reference frame (or
-                    // S0) into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
-                    fscal[c] = ci == 0 ? expf(gref[e])
-                                       : expf(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref[e]);
-                    scal[buf * 128 + c] = gref[e];
-                    scal[256 + buf * 128 + c] = glast[e];
-                }
-            }
-            // X = w (.) v tiles (their space holds nothing raw)
-#pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
-                float vf[4], wf[4];
-                unpack4_bf16(vq[pss], vf);
-                unpack4_bf16(wq[pss], wf);
-                uint2 xh, xl;
-                split2(wf[0] * vf[0], wf[1] * vf[1], xh.x, xl.x);
-                split2(wf[2] * vf[2], wf[3] * vf[3], xh.y, xl.y);
-                const uint32_t o = off_rowmajor(i, c0);
-                *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
-                *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
+            bar_sync_1<NS>();
+            if (tid < D) {
+                const int c = tid;
+                const float glast = htot[c] + htot[128 + c];
+                const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
+                // factor taking the state from the previous chunk's reference frame (or S0)
+                // into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
+                fscal[c] = ci == 0 ? expf(gref) : expf(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref);
+                scal[buf * 128 + c] = gref;
+                scal[256 + buf * 128 + c] = glast;
             }
             // group B: q, k, b; the tiles below overwrite these rows and the staged o tile
             uint2 qq[8], kq[8], bq[8];
@@ -333,13 +405,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
             }
             if (tid == 0) bulk_wait_read0();
-            if (__syncthreads_or(fault)) {
+            if (bar_or_1<NS>(fault)) {
                 fault = true;
                 break;
             }
+            // G - Gref for tokens 0..31; tokens 32..63 add the lower half's total
+            const float4 gr4 = *reinterpret_cast<const float4*>(scal + buf * 128 + c0);
+            const float4 ht4 = *reinterpret_cast<const float4*>(htot + c0);
+            const float glo[4] = {-gr4.x, -gr4.y, -gr4.z, -gr4.w};
+            const float ghi[4] = {ht4.x - gr4.x, ht4.y - gr4.y, ht4.z - gr4.z, ht4.w - gr4.w};
 #pragma unroll
             for (int pss = 0; pss < 8; ++pss) {
                 const int i = 8 * pss + tl;
+                const float4 g4 = *reinterpret_cast<const float4*>(smem + OFF_RAW_LA + raw_off_f32(i, c0));
+                const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
                 float qf[4], kf[4], bf[4];
                 unpack4_bf16(qq[pss], qf);
                 unpack4_bf16(kq[pss], kf);
@@ -349,8 +428,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 for (int e = 0; e < 4; ++e) {
                     // fast exponential: relative error a few 1e-6 for |arguments| up to ~45,
                     // well below the 2^-16 carried by the hi/lo operand splits
-                    const float ge = __expf(G[pss][e] - gref[e]);
-                    const float gi = __expf(gref[e] - G[pss][e]);
+                    const float d = gv[e] + (pss < 4 ? glo[e] : ghi[e]);  // G - Gref
+                    const float ge = __expf(d);
+                    const float gi = __expf(-d);
                     kh[e] = kf[e] * ge;
                     qv[e] = qf[e] * ge;
                     kb[e] = kf[e] * gi;
@@ -371,33 +451,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         fence_proxy_async_smem();
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
 
         // ------------------------------------------------------------ 2. Gram MMAs
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id128 = idesc_bf16(128, 128, false, false);
-            const uint32_t id64 = idesc_bf16(128, 64, false, false);
+        if (tid == 0) mbar_arrive(mbar(RDY_G));
+        // X = w (.) v tiles while the Gram MMAs run (their space holds nothing raw; the
+        // epilogue below overwrites the raw v / w rows, after the next barrier)
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t kofs = ks * 256;
-                mma_bf16(tmem + TM_G, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
-                         sdesc(sbase + OFF_KH + kofs, 128, 2048), id128, ks > 0);
-            }
-            mma_commit(mbar(MB_G));
-            // P cross terms (lanes 0..63 hold Kb rows; lanes 64..127 are masked out)
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t kofs = ks * 256;
-                mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBL + kofs, 128, 2048),
-                         sdesc(sbase + OFF_QH + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
-                mma_bf16(tmem + TM_G + 64, sdesc(sbase + OFF_KBH + kofs, 128, 2048),
-                         sdesc(sbase + OFF_QL + kofs, 128, 2048), id64, 1u, 0u, 0u, 0xffffffffu, 0xffffffffu);
-            }
-            mma_commit(mbar(MB_GX));
+        for (int pss = 0; pss < 8; ++pss) {
+            const int i = 8 * pss + tl;
+            const bool valid = i < nvalid;
+            const uint32_t ro = raw_off_bf16(i, c0);
+            const uint2 z = make_uint2(0u, 0u);
+            float vf[4], wf[4];
+            unpack4_bf16(valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_V + ro) : z, vf);
+            unpack4_bf16(valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_W + ro) : z, wf);
+            uint2 xh, xl;
+            split2(wf[0] * vf[0], wf[1] * vf[1], xh.x, xl.x);
+            split2(wf[2] * vf[2], wf[3] * vf[3], xh.y, xl.y);
+            const uint32_t o = off_rowmajor(i, c0);
+            *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
+            *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
         }
         fault |= !mbar_wait(mbar(MB_G), par, kWaitNs);
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
 
         // ------------------------------------------------------------ 3. Gram epilogue
@@ -451,23 +528,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
 
         // ------------------------------------------------------------ 4. D1 = X^T [B;P]^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id128 = idesc_bf16(128, 128, true, true);
-            const uint32_t id64 = idesc_bf16(128, 64, true, true);
-#pragma unroll
-            for (int ks = 0; ks < CH / 16; ++ks) {
-                const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
-                const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
-                mma_bf16(tmem + TM_D1, xh, sdesc(sbase + OFF_B + ks * 256, 128, 1024), id128, ks > 0);
-                mma_bf16(tmem + TM_D1 + 64, xl, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
-                mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PL + ks * 256, 128, 1024), id64, 1u);
-            }
-            mma_commit(mbar(MB_2B));
-        }
+        if (tid == 0) mbar_arrive(mbar(RDY_2B));
         // ------------------------------------------------------------ 5. state epilogue
         {
             uint32_t packed[32];
@@ -483,9 +547,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     }
                 } else {
                     tmem_ld32(tmem + lane_bits + TM_U + cb, u);
+                    const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] *= fscal[cb + e];
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 f = f4[e4];
+                        u[4 * e4] *= f.x;
+                        u[4 * e4 + 1] *= f.y;
+                        u[4 * e4 + 2] *= f.z;
+                        u[4 * e4 + 3] *= f.w;
+                    }
                 }
                 tmem_st32(tmem + lane_bits + TM_U + cb, u);
 #pragma unroll
@@ -499,21 +570,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             tmem_wait_st();
         }
         tc_fence_before();
-        __syncthreads();
+        bar_sync_1<NS>();
 
         // ------------------------------------------------------------ 6. D1 += Sref^T [Kh;Qh]^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id128 = idesc_bf16(128, 128, false, false);
-            const uint32_t id64 = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const uint32_t a = tmem + TM_S + ks * 8;
-                mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
-                mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
-            }
-            mma_commit(mbar(MB_2A));
-        }
+        if (tid == 0) mbar_arrive(mbar(RDY_2A));
         // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
         // The next chunk's q, k, b may land over Kh / Qh / Ql as soon as the Sref MMAs are
         // done; thread 0 checks between the solve's levels and issues them then.
@@ -530,32 +590,27 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
         // (the same row for a whole warp: broadcast), columns as consecutive floats.
         if (tid < 64) {
+            // column jj of block bI, right-looking: once x_l is final, every later row takes
+            // its term, so the chain from one row to the next is a single FMA
             const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
+            const float* ablk = WA + 16 * bI * WS + 16 * bI;
             float x[16];
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float* arow = WA + (16 * bI + r) * WS + 16 * bI;
-                float s = 0.f;
+            for (int r = 0; r < 16; ++r) x[r] = 0.f;
 #pragma unroll
-                for (int l4 = 0; l4 < 16; l4 += 4) {
-                    if (l4 < r) {
-                        const float4 a = *reinterpret_cast<const float4*>(arow + l4);
-                        const float av[4] = {a.x, a.y, a.z, a.w};
+            for (int l = 0; l < 16; ++l) {
+                x[l] = l < jj ? 0.f : (l == jj ? 1.f : x[l]);
+                WT[(16 * bI + l) * WS + col] = x[l];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (l4 + u < r) s += (l4 + u >= jj) ? av[u] * x[l4 + u] : 0.f;
-                    }
-                }
-                x[r] = (r < jj) ? 0.f : (r == jj ? 1.f : -s);
-                WT[(16 * bI + r) * WS + col] = x[r];
+                for (int r = l + 1; r < 16; ++r) x[r] = fmaf(-ablk[r * WS + l], x[l], x[r]);
             }
         } else {
-            for (int idx = tid - 64; idx < 64 * 64; idx += NT - 64) {
+            for (int idx = tid - 64; idx < 64 * 64; idx += NS - 64) {
                 const int r = idx >> 6, c = idx & 63;
                 if ((c >> 4) > (r >> 4)) WT[r * WS + c] = 0.f;
             }
         }
-        __syncthreads();
+        bar_sync_1<NS>();
         try_issue_raw_b();
         {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
             const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
@@ -577,7 +632,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             WM[((tid >> 7) * 16 + r0) * 33 + c] = m0;
             WM[((tid >> 7) * 16 + r0 + 8) * 33 + c] = m1;
         }
-        __syncthreads();
+        bar_sync_1<NS>();
         {   // level 2, step 2: T_10 = -T_11 M
             const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
             const float* Mb = WM + (tid >> 7) * 16 * 33;
@@ -599,7 +654,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             WT[(base + 16 + r0) * WS + base + c] = -t0;
             WT[(base + 24 + r0) * WS + base + c] = -t1;
         }
-        __syncthreads();
+        bar_sync_1<NS>();
         try_issue_raw_b();
         {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
             const int c = tid & 31, r0 = tid >> 5;
@@ -618,7 +673,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
             for (int k = 0; k < 4; ++k) WM[(r0 + 8 * k) * 33 + c] = m[k];
         }
-        __syncthreads();
+        bar_sync_1<NS>();
         {   // level 3, step 2: T_BA = -T_BB M (T_BB lower triangular, its upper part is zero)
             const int c = tid & 31, r0 = tid >> 5;
             float t[4] = {0.f, 0.f, 0.f, 0.f};
@@ -636,18 +691,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
             for (int k = 0; k < 4; ++k) WT[(32 + r0 + 8 * k) * WS + c] = -t[k];
         }
-        __syncthreads();
-        for (int idx = tid; idx < 512; idx += NT) {  // T as a K-major bf16 B operand [i][j]
+        bar_sync_1<NS>();
+        for (int idx = tid; idx < 512; idx += NS) {  // T as a K-major bf16 B operand [i][j]
             const int i = idx & 63, jg = idx >> 6;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        bar_sync_1<NS>();
 
         fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
         if (tid == 0 && ci + 1 < nchunks) {
             issue_raw_a(tc0 + CH);                   // B / P and the solve's workspace are dead
@@ -662,25 +717,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(y[2 * e], y[2 * e + 1]);
-            __syncthreads();  // every half has read its fp32 columns before any are overwritten
+            bar_sync_1<NS>();  // every half has read its fp32 columns before any are overwritten
             tmem_st16(tmem + lane_bits + TM_D1 + 16 * hf, pk);
             tmem_wait_st();
         }
         tc_fence_before();
-        __syncthreads();
+        bar_sync_1<NS>();
 
         // ------------------------------------------------------------ 8. R^T = Y^T T^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id64 = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int ks = 0; ks < CH / 16; ++ks)
-                mma_bf16_ts(tmem + TM_R, tmem + TM_D1 + ks * 8, sdesc(sbase + OFF_T + ks * 2048, 1024, 128), id64,
-                            ks > 0);
-            mma_commit(mbar(MB_3));
-        }
+        if (tid == 0) mbar_arrive(mbar(RDY_3));
         fault |= !mbar_wait(mbar(MB_3), par, kWaitNs);
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
 
         // ------------------------------------------------------------ 9. -R^T as a bf16 A operand
@@ -691,34 +738,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             uint32_t pk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(-r[2 * e], -r[2 * e + 1]);
-            __syncthreads();  // every half has read its fp32 columns before any are overwritten
+            bar_sync_1<NS>();  // every half has read its fp32 columns before any are overwritten
             tmem_st16(tmem + lane_bits + TM_R + 16 * hf, pk);
             tmem_wait_st();
         }
         tc_fence_before();
-        __syncthreads();
+        bar_sync_1<NS>();
 
         // ------------------------------------------------------------ 10. output and state MMAs
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id_o = idesc_bf16(128, 64, false, true);
-            const uint32_t id_xx = idesc_bf16(128, 128, true, true);
-            const uint32_t id_rx = idesc_bf16(128, 128, false, true);
-#pragma unroll
-            for (int ks = 0; ks < CH / 16; ++ks) {
-                const uint32_t rr = tmem + TM_R + ks * 8;
-                const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
-                const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
-                mma_bf16_ts(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
-                mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
-                mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
-                mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
-                mma_bf16_ts(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
-            }
-            mma_commit(mbar(MB_45));
-        }
+        if (tid == 0) mbar_arrive(mbar(RDY_45));
         fault |= !mbar_wait(mbar(MB_45), par, kWaitNs);
-        if (__syncthreads_or(fault)) { fault = true; break; }
+        if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
 
         // ------------------------------------------------------------ 11. o
@@ -732,7 +762,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 32; ++e) ost[(32 * hf + e) * D + L] = ov[e];
                 fence_proxy_async_smem();
-                __syncthreads();
+                bar_sync_1<NS>();
                 if (tid == 0) {
                     tma_store_3d(&maps.o, sbase + OFF_OST, 0, h, tc0);
                     bulk_commit();
@@ -746,12 +776,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         tc_fence_before();
-        __syncthreads();
+        bar_sync_1<NS>();
     }
     // the staged o tile must be read out before shared memory is released or rewritten
     if (tid == 0) bulk_wait_read0();
 
-    if (!fault && p.S_T) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
+    if (!fault && p.S_T && warp != kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
         tc_fence_after();
 #pragma unroll
@@ -767,7 +797,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
     }
-    if (fault && tid == 0) atomicOr(&g_tc_fault, 1u);
+    if (fault && (tid == 0 || tid == NS)) atomicOr(&g_tc_fault, 1u);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);

@@ -89,6 +89,37 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64
     }
 }
 
+// The value unchanged, but opaque to the optimiser (which can then neither fold nor hoist
+// what is computed from it).
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
+    asm volatile("" : "+r"(v));
+    return v;
+}
+
+// One arrival (release semantics at CTA scope) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
+// Named barrier 1 over the first `count` threads of the CTA (a multiple of 32); barrier 0
+// stays the whole-CTA __syncthreads.
+template <int count>
+__device__ __forceinline__ void bar_sync_1() {
+    asm volatile("bar.sync 1, %0;" ::"n"(count) : "memory");
+}
+
+// Named barrier 1 over `count` threads that also returns the OR of `v` across them.
+template <int count>
+__device__ __forceinline__ bool bar_or_1(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, 1, %2, p;\nselp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(count)
+        : "memory");
+    return r != 0;
+}
+
 // Non-blocking: has the phase with the given parity completed?
 __device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
     uint32_t ok;
