@@ -24,10 +24,13 @@
 // significant bits); Qh Sref splits Qh only (Qh_hi Sref + Qh_lo Sref); the erase path
 // (A, B, Qm, T, Y, R) stays in plain bf16.
 //
-// Phases per chunk. Eight SIMT warps take part in each (thread t serves tensor-memory lane
-// t % 128 and column half t / 128); a ninth warp only issues the MMA groups, each as soon
-// as the SIMT warps signal that its operands are written, so no SIMT warp waits behind the
-// tensor pipe. The MMAs of phases 4 and 6 run while the UT solve's SIMT work proceeds:
+// Phases per chunk. Sixteen SIMT warps take part in each (thread t serves tensor-memory
+// lane t % 128 and column quarter t / 128): the phases are chains of dependent
+// shared-memory, tensor-memory and special-function operations, and four warps per
+// scheduler hide their latency where two did not. A seventeenth warp only issues the MMA
+// groups, each as soon as the SIMT warps signal that its operands are written, so no SIMT
+// warp waits behind the tensor pipe. The MMAs of phases 4 and 6 run while the UT solve's
+// SIMT work proceeds:
 //   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
 //             written while they run
@@ -54,8 +57,8 @@ using namespace tc;
 
 constexpr int CH = 64;   // chunk length
 constexpr int D = 128;   // dk = dv
-constexpr int NS = 256;           // SIMT threads (warps 0..7): prep, epilogues, solve
-constexpr int kIssuer = NS / 32;  // warp 8 issues every MMA
+constexpr int NS = 512;           // SIMT threads (warps 0..15): prep, epilogues, solve
+constexpr int kIssuer = NS / 32;  // warp 16 issues every MMA
 constexpr int NT = NS + 32;       // threads per CTA
 constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
 
@@ -100,9 +103,9 @@ constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
 constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
 constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
-// float gref[2][128], glast[2][128], f[128], half-chunk log-decay totals [2][128]
+// float gref[2][128], glast[2][128], f[128], quarter-chunk log-decay totals [4][128]
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
-constexpr uint32_t OFF_MBAR = OFF_SCAL + 7 * 128 * 4;
+constexpr uint32_t OFF_MBAR = OFF_SCAL + 9 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 16 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
 static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
@@ -183,12 +186,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int L = tid & 127;   // tensor-memory lane served by this thread
-    const int hf = tid >> 7;   // column half
+    const int cp = tid >> 7;   // column quarter (SIMT threads)
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
     float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast
     float* fscal = scal + 512;                                  // [128] state frame factors
-    float* htot = scal + 640;  // [2][128] sums of log_alpha over tokens 0..31 and 32..63
+    float* qtot = scal + 640;  // [4][128] sums of log_alpha over tokens 16q .. 16q + 15
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
     float* WT = reinterpret_cast<float*>(smem + OFF_WT);
     float* WM = reinterpret_cast<float*>(smem + OFF_WM);
@@ -223,9 +226,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT);
     bool fault = false;
 
-    // prep mapping: warp w owns channels [16w, 16w+16); lane = (channel quad, token in block)
-    const int tl = lane & 7;
-    const int c0 = 16 * warp + 4 * (lane >> 3);
+    // prep mapping: warp w owns channels [16(w % 8), +16) and tokens [32 th, +32) with
+    // th = w / 8; lane = (channel quad, token in a block of 8)
+    const int th = (warp >> 3) & 1;
+    const int ti0 = 32 * th + (lane & 7);
+    const int c0 = 16 * (warp & 7) + 4 * (lane >> 3);
 
     // raw inputs of a chunk in two groups, each issued as soon as its space frees up
     auto issue_raw_a = [&](int ts) {  // log_alpha, v, w
@@ -365,25 +370,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             // group A: log_alpha, v, w (tokens past the sequence end count as zero); v and w
             // are read after the Gram MMAs are under way.
             // Cumulative log-decay G, in place over the staged log_alpha rows: thread
-            // (channel c, half hh) sums tokens 32hh .. 32hh + 31 of channel c. The upper half
-            // still lacks the lower half's total, which is added where G is read.
+            // (channel c, quarter cp) sums tokens 16cp .. 16cp + 15 of channel c. The totals
+            // of the earlier quarters are added where G is read.
             fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
             {
-                const int c = tid & 127, hh = tid >> 7;
+                const int c = L;
                 float acc = 0.f;
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    const int i = 32 * hh + r;
+                for (int r = 0; r < 16; ++r) {
+                    const int i = 16 * cp + r;
                     float* gp = reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c));
                     acc += i < nvalid ? *gp : 0.f;
                     *gp = acc;
                 }
-                htot[128 * hh + c] = acc;
+                qtot[128 * cp + c] = acc;
             }
             bar_sync_1<NS>();
             if (tid < D) {
                 const int c = tid;
-                const float glast = htot[c] + htot[128 + c];
+                const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
                 const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
                 // factor taking the state from the previous chunk's reference frame (or S0)
                 // into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
@@ -392,11 +397,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 scal[256 + buf * 128 + c] = glast;
             }
             // group B: q, k, b; the tiles below overwrite these rows and the staged o tile
-            uint2 qq[8], kq[8], bq[8];
+            uint2 qq[4], kq[4], bq[4];
             fault |= !mbar_wait(mbar(MB_RAWB), par, kWaitNs);
 #pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
+            for (int pss = 0; pss < 4; ++pss) {
+                const int i = ti0 + 8 * pss;
                 const bool valid = i < nvalid;
                 const uint32_t o = raw_off_bf16(i, c0);
                 const uint2 z = make_uint2(0u, 0u);
@@ -409,14 +414,22 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 fault = true;
                 break;
             }
-            // G - Gref for tokens 0..31; tokens 32..63 add the lower half's total
-            const float4 gr4 = *reinterpret_cast<const float4*>(scal + buf * 128 + c0);
-            const float4 ht4 = *reinterpret_cast<const float4*>(htot + c0);
-            const float glo[4] = {-gr4.x, -gr4.y, -gr4.z, -gr4.w};
-            const float ghi[4] = {ht4.x - gr4.x, ht4.y - gr4.y, ht4.z - gr4.z, ht4.w - gr4.w};
+            // G - Gref: this thread's tokens lie in quarters 2th and 2th + 1, whose offsets
+            // are the totals of the quarters before them
+            float dlo[4], dhi[4];
+            {
+                const float4 gr4 = *reinterpret_cast<const float4*>(scal + buf * 128 + c0);
+                const float gr[4] = {gr4.x, gr4.y, gr4.z, gr4.w};
 #pragma unroll
-            for (int pss = 0; pss < 8; ++pss) {
-                const int i = 8 * pss + tl;
+                for (int e = 0; e < 4; ++e) {
+                    const float t0q = qtot[c0 + e], t1q = qtot[128 + c0 + e], t2q = qtot[256 + c0 + e];
+                    dlo[e] = (th ? t0q + t1q : 0.f) - gr[e];
+                    dhi[e] = (th ? (t0q + t1q) + t2q : t0q) - gr[e];
+                }
+            }
+#pragma unroll
+            for (int pss = 0; pss < 4; ++pss) {
+                const int i = ti0 + 8 * pss;
                 const float4 g4 = *reinterpret_cast<const float4*>(smem + OFF_RAW_LA + raw_off_f32(i, c0));
                 const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
                 float qf[4], kf[4], bf[4];
@@ -428,7 +441,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 for (int e = 0; e < 4; ++e) {
                     // fast exponential: relative error a few 1e-6 for |arguments| up to ~45,
                     // well below the 2^-16 carried by the hi/lo operand splits
-                    const float d = gv[e] + (pss < 4 ? glo[e] : ghi[e]);  // G - Gref
+                    const float d = gv[e] + (pss < 2 ? dlo[e] : dhi[e]);  // G - Gref
                     const float ge = __expf(d);
                     const float gi = __expf(-d);
                     kh[e] = kf[e] * ge;
@@ -458,8 +471,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // X = w (.) v tiles while the Gram MMAs run (their space holds nothing raw; the
         // epilogue below overwrites the raw v / w rows, after the next barrier)
 #pragma unroll
-        for (int pss = 0; pss < 8; ++pss) {
-            const int i = 8 * pss + tl;
+        for (int pss = 0; pss < 4; ++pss) {
+            const int i = ti0 + 8 * pss;
             const bool valid = i < nvalid;
             const uint32_t ro = raw_off_bf16(i, c0);
             const uint2 z = make_uint2(0u, 0u);
@@ -478,51 +491,51 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_after();
 
         // ------------------------------------------------------------ 3. Gram epilogue
+        // Thread (lane L, quarter cp) takes Gram columns 32cp .. 32cp + 31: lanes 0..63 are
+        // Kb rows (B, then P), lanes 64..127 Eb rows (A, then Qm); column i, row j = L % 64.
         {
-            // warps 4..7 on lanes 0..63 read the P block, which the cross terms still update
-            if (hf == 1 && L < 64) {
+            // lanes 0..63 of the P block: the cross terms still update it
+            if (cp >= 2 && L < 64) {
                 if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
                 tc_fence_after();
             }
-            float v0[32], v1[32];
-            tmem_ld32(tmem + lane_bits + TM_G + 64 * hf, v0);
-            tmem_ld32(tmem + lane_bits + TM_G + 64 * hf + 32, v1);
-            tmem_wait_ld();
+            float v[32];
+            tmem_ld32_wait(tmem + lane_bits + TM_G + 32 * cp, v);
             const int j = L & 63;
-            auto val = [&](int i) { return i < 32 ? v0[i] : v1[i - 32]; };
-            if (L < 64 && hf == 0) {  // B_ij, j < i
+            const int ib = 32 * (cp & 1);  // first i of this thread
+            if (L < 64 && cp < 2) {  // B_ij, j < i
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) {
+                for (int q = 0; q < 4; ++q) {
                     float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = (8 * q8 + e > j) ? val(8 * q8 + e) : 0.f;
-                    store8_bf16(smem, OFF_B + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
+                    for (int e = 0; e < 8; ++e) f[e] = (ib + 8 * q + e > j) ? v[8 * q + e] : 0.f;
+                    store8_bf16(smem, OFF_B + (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
                 }
             } else if (L < 64) {  // P_ij, j <= i, split hi / lo (after the cross terms)
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) {
+                for (int q = 0; q < 4; ++q) {
                     float x[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
+                    for (int e = 0; e < 8; ++e) x[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
                     uint4 hi, lo;
                     split2(x[0], x[1], hi.x, lo.x);
                     split2(x[2], x[3], hi.y, lo.y);
                     split2(x[4], x[5], hi.z, lo.z);
                     split2(x[6], x[7], hi.w, lo.w);
-                    const uint32_t o = q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16;
+                    const uint32_t o = (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16;
                     *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
                     *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
                 }
-            } else if (hf == 0) {  // A_ij, j < i, fp32 for the solve
+            } else if (cp < 2) {  // A_ij, j < i, fp32 for the solve
 #pragma unroll
-                for (int i = 0; i < 64; ++i) WA[i * WS + j] = (i > j) ? val(i) : 0.f;
+                for (int e = 0; e < 32; ++e) WA[(ib + e) * WS + j] = (ib + e > j) ? v[e] : 0.f;
             } else {  // Qm_ij, j <= i
 #pragma unroll
-                for (int q8 = 0; q8 < 8; ++q8) {
+                for (int q = 0; q < 4; ++q) {
                     float f[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = (8 * q8 + e >= j) ? val(8 * q8 + e) : 0.f;
-                    store8_bf16(smem, OFF_QM + q8 * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
+                    for (int e = 0; e < 8; ++e) f[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
+                    store8_bf16(smem, OFF_QM + (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
                 }
             }
         }
@@ -533,40 +546,34 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // ------------------------------------------------------------ 4. D1 = X^T [B;P]^T
         if (tid == 0) mbar_arrive(mbar(RDY_2B));
         // ------------------------------------------------------------ 5. state epilogue
+        // Thread (lane L, quarter cp) takes key channels 32cp .. 32cp + 31.
         {
-            uint32_t packed[32];
+            const int cb = 32 * cp;
+            float u[32];
+            if (ci == 0) {
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int cb = 64 * hf + 32 * part;
-                float u[32];
-                if (ci == 0) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = cb + e;
-                        u[e] = (p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f) * fscal[c];
-                    }
-                } else {
-                    tmem_ld32(tmem + lane_bits + TM_U + cb, u);
-                    const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 f = f4[e4];
-                        u[4 * e4] *= f.x;
-                        u[4 * e4 + 1] *= f.y;
-                        u[4 * e4 + 2] *= f.z;
-                        u[4 * e4 + 3] *= f.w;
-                    }
+                for (int e = 0; e < 32; ++e) {
+                    const int c = cb + e;
+                    u[e] = (p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f) * fscal[c];
                 }
-                tmem_st32(tmem + lane_bits + TM_U + cb, u);
+            } else {
+                tmem_ld32_wait(tmem + lane_bits + TM_U + cb, u);
+                const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) packed[16 * part + e] = pack_bf16(u[2 * e], u[2 * e + 1]);
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 f = f4[e4];
+                    u[4 * e4] *= f.x;
+                    u[4 * e4 + 1] *= f.y;
+                    u[4 * e4 + 2] *= f.z;
+                    u[4 * e4 + 3] *= f.w;
+                }
             }
-            // Sref^T as a bf16 A operand: key channels 64*hf .. +63 in columns 32*hf .. +31
-            float pk[32];
+            tmem_st32(tmem + lane_bits + TM_U + cb, u);
+            // Sref^T as a bf16 A operand: key channels cb .. cb + 31 in columns cb/2 .. +15
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) pk[e] = __uint_as_float(packed[e]);
-            tmem_st32(tmem + lane_bits + TM_S + 32 * hf, pk);
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(u[2 * e], u[2 * e + 1]);
+            tmem_st16(tmem + lane_bits + TM_S + 16 * cp, pk);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -588,7 +595,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
         // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
         // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
-        // (the same row for a whole warp: broadcast), columns as consecutive floats.
+        // (the same row for many lanes: broadcast), columns as consecutive floats.
         if (tid < 64) {
             // column jj of block bI, right-looking: once x_l is final, every later row takes
             // its term, so the chain from one row to the next is a single FMA
@@ -612,88 +619,76 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         bar_sync_1<NS>();
         try_issue_raw_b();
-        {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 2 per thread)
-            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
-            const float* a0 = WA + (base + 16 + r0) * WS + base;
-            const float* a1 = WA + (base + 24 + r0) * WS + base;
-            float m0 = 0.f, m1 = 0.f;
+        {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 1 per thread)
+            const int blk = tid >> 8, base = 32 * blk, r = (tid >> 4) & 15, c = tid & 15;
+            const float* a0 = WA + (base + 16 + r) * WS + base;
+            float m = 0.f;
 #pragma unroll
             for (int l4 = 0; l4 < 16; l4 += 4) {
                 const float4 x0 = *reinterpret_cast<const float4*>(a0 + l4);
-                const float4 x1 = *reinterpret_cast<const float4*>(a1 + l4);
-                const float xa[4] = {x0.x, x0.y, x0.z, x0.w}, xb[4] = {x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float t = WT[(base + l4 + u) * WS + base + c];
-                    m0 += xa[u] * t;
-                    m1 += xb[u] * t;
-                }
+                m = fmaf(x0.x, WT[(base + l4) * WS + base + c], m);
+                m = fmaf(x0.y, WT[(base + l4 + 1) * WS + base + c], m);
+                m = fmaf(x0.z, WT[(base + l4 + 2) * WS + base + c], m);
+                m = fmaf(x0.w, WT[(base + l4 + 3) * WS + base + c], m);
             }
-            WM[((tid >> 7) * 16 + r0) * 33 + c] = m0;
-            WM[((tid >> 7) * 16 + r0 + 8) * 33 + c] = m1;
+            WM[(blk * 16 + r) * 33 + c] = m;
         }
         bar_sync_1<NS>();
         {   // level 2, step 2: T_10 = -T_11 M
-            const int base = 32 * (tid >> 7), c = tid & 15, r0 = (tid >> 4) & 7;
-            const float* Mb = WM + (tid >> 7) * 16 * 33;
-            const float* t0r = WT + (base + 16 + r0) * WS + base + 16;
-            const float* t1r = WT + (base + 24 + r0) * WS + base + 16;
-            float t0 = 0.f, t1 = 0.f;
+            const int blk = tid >> 8, base = 32 * blk, r = (tid >> 4) & 15, c = tid & 15;
+            const float* Mb = WM + blk * 16 * 33;
+            const float* t0r = WT + (base + 16 + r) * WS + base + 16;
+            float t = 0.f;
 #pragma unroll
             for (int l4 = 0; l4 < 16; l4 += 4) {
-                const float4 y0 = *reinterpret_cast<const float4*>(t0r + l4);
-                const float4 y1 = *reinterpret_cast<const float4*>(t1r + l4);
-                const float ya[4] = {y0.x, y0.y, y0.z, y0.w}, yb[4] = {y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float mv = Mb[(l4 + u) * 33 + c];
-                    t0 += ya[u] * mv;  // T_11's upper triangle is stored as zeros
-                    t1 += yb[u] * mv;
-                }
+                const float4 y0 = *reinterpret_cast<const float4*>(t0r + l4);  // upper triangle: zeros
+                t = fmaf(y0.x, Mb[(l4) * 33 + c], t);
+                t = fmaf(y0.y, Mb[(l4 + 1) * 33 + c], t);
+                t = fmaf(y0.z, Mb[(l4 + 2) * 33 + c], t);
+                t = fmaf(y0.w, Mb[(l4 + 3) * 33 + c], t);
             }
-            WT[(base + 16 + r0) * WS + base + c] = -t0;
-            WT[(base + 24 + r0) * WS + base + c] = -t1;
+            WT[(base + 16 + r) * WS + base + c] = -t;
         }
         bar_sync_1<NS>();
         try_issue_raw_b();
-        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 4 outputs per thread)
+        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 2 outputs per thread)
             const int c = tid & 31, r0 = tid >> 5;
-            float m[4] = {0.f, 0.f, 0.f, 0.f};
+            float m[2] = {0.f, 0.f};
 #pragma unroll
             for (int l4 = 0; l4 < 32; l4 += 4) {
                 float tv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) tv[u] = WT[(l4 + u) * WS + c];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 a = *reinterpret_cast<const float4*>(WA + (32 + r0 + 8 * k) * WS + l4);
+                for (int k = 0; k < 2; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WA + (32 + r0 + 16 * k) * WS + l4);
                     m[k] += a.x * tv[0] + a.y * tv[1] + a.z * tv[2] + a.w * tv[3];
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) WM[(r0 + 8 * k) * 33 + c] = m[k];
+            for (int k = 0; k < 2; ++k) WM[(r0 + 16 * k) * 33 + c] = m[k];
         }
         bar_sync_1<NS>();
         {   // level 3, step 2: T_BA = -T_BB M (T_BB lower triangular, its upper part is zero)
             const int c = tid & 31, r0 = tid >> 5;
-            float t[4] = {0.f, 0.f, 0.f, 0.f};
+            float t[2] = {0.f, 0.f};
 #pragma unroll
             for (int l4 = 0; l4 < 32; l4 += 4) {
                 float mv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) mv[u] = WM[(l4 + u) * 33 + c];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float4 a = *reinterpret_cast<const float4*>(WT + (32 + r0 + 8 * k) * WS + 32 + l4);
+                for (int k = 0; k < 2; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WT + (32 + r0 + 16 * k) * WS + 32 + l4);
                     t[k] += a.x * mv[0] + a.y * mv[1] + a.z * mv[2] + a.w * mv[3];
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) WT[(32 + r0 + 8 * k) * WS + c] = -t[k];
+            for (int k = 0; k < 2; ++k) WT[(32 + r0 + 16 * k) * WS + c] = -t[k];
         }
         bar_sync_1<NS>();
-        for (int idx = tid; idx < 512; idx += NS) {  // T as a K-major bf16 B operand [i][j]
-            const int i = idx & 63, jg = idx >> 6;
+        {   // T as a K-major bf16 B operand [i][j]
+            const int i = tid & 63, jg = tid >> 6;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
         }
         fence_proxy_async_smem();
@@ -710,15 +705,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
 
         // ------------------------------------------------------------ 7. Y^T as a bf16 A operand
+        // Thread (lane L, quarter cp) takes tokens 16cp .. 16cp + 15 (fp32 columns), packed
+        // into columns 8cp .. 8cp + 7.
         {
-            float y[32];
-            tmem_ld32(tmem + lane_bits + TM_D1 + 32 * hf, y);
-            tmem_wait_ld();
-            uint32_t pk[16];
+            float y[16];
+            tmem_ld16_wait(tmem + lane_bits + TM_D1 + 16 * cp, y);
+            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(y[2 * e], y[2 * e + 1]);
-            bar_sync_1<NS>();  // every half has read its fp32 columns before any are overwritten
-            tmem_st16(tmem + lane_bits + TM_D1 + 16 * hf, pk);
+            for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(y[2 * e], y[2 * e + 1]);
+            bar_sync_1<NS>();  // every quarter has read its fp32 columns before any are overwritten
+            tmem_st8(tmem + lane_bits + TM_D1 + 8 * cp, pk);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -732,14 +728,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 9. -R^T as a bf16 A operand
         {
-            float r[32];
-            tmem_ld32(tmem + lane_bits + TM_R + 32 * hf, r);
-            tmem_wait_ld();
-            uint32_t pk[16];
+            float r[16];
+            tmem_ld16_wait(tmem + lane_bits + TM_R + 16 * cp, r);
+            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(-r[2 * e], -r[2 * e + 1]);
-            bar_sync_1<NS>();  // every half has read its fp32 columns before any are overwritten
-            tmem_st16(tmem + lane_bits + TM_R + 16 * hf, pk);
+            for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(-r[2 * e], -r[2 * e + 1]);
+            bar_sync_1<NS>();  // every quarter has read its fp32 columns before any are overwritten
+            tmem_st8(tmem + lane_bits + TM_R + 8 * cp, pk);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -752,15 +747,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_after();
 
         // ------------------------------------------------------------ 11. o
+        // Thread (lane L = value channel, quarter cp) takes tokens 16cp .. 16cp + 15.
         {
-            float ov[32];
-            tmem_ld32(tmem + lane_bits + TM_D1 + 64 + 32 * hf, ov);
-            tmem_wait_ld();
+            float ov[16];
+            tmem_ld16_wait(tmem + lane_bits + TM_D1 + 64 + 16 * cp, ov);
             if (kTmaStoreO<TO> && nvalid == CH) {
                 // stage the fp32 tile [token][channel] and let one TMA store write it
                 float* ost = reinterpret_cast<float*>(smem + OFF_OST);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ost[(32 * hf + e) * D + L] = ov[e];
+                for (int e = 0; e < 16; ++e) ost[(16 * cp + e) * D + L] = ov[e];
                 fence_proxy_async_smem();
                 bar_sync_1<NS>();
                 if (tid == 0) {
@@ -769,8 +764,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int i = 32 * hf + e;
+                for (int e = 0; e < 16; ++e) {
+                    const int i = 16 * cp + e;
                     if (i < nvalid) op[((size_t)(tc0 + i) * p.h_v + h) * D + L] = from_f32<TO>(ov[e]);
                 }
             }
@@ -784,17 +779,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     if (!fault && p.S_T && warp != kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
         tc_fence_after();
+        const int cb = 32 * cp;
+        float u[32];
+        tmem_ld32_wait(tmem + lane_bits + TM_U + cb, u);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int cb = 64 * hf + 32 * part;
-            float u[32];
-            tmem_ld32(tmem + lane_bits + TM_U + cb, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int c = cb + e;
-                p.S_T[soff + (size_t)c * D + L] = u[e] * expf(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
-            }
+        for (int e = 0; e < 32; ++e) {
+            const int c = cb + e;
+            p.S_T[soff + (size_t)c * D + L] = u[e] * expf(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
         }
     }
     if (fault && (tid == 0 || tid == NS)) atomicOr(&g_tc_fault, 1u);
