@@ -29,8 +29,9 @@
 // shared-memory, tensor-memory and special-function operations, and four warps per
 // scheduler hide their latency where two did not. A seventeenth warp only issues the MMA
 // groups, each as soon as the SIMT warps signal that its operands are written, so no SIMT
-// warp waits behind the tensor pipe. The MMAs of phases 4 and 6 run while the UT solve's
-// SIMT work proceeds:
+// warp waits behind the tensor pipe; an eighteenth issues the TMA loads of the next chunk's
+// raw rows as soon as their space is free. The MMAs of phases 4 and 6 run while the UT
+// solve's SIMT work proceeds:
 //   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
 //             written while they run
@@ -58,8 +59,9 @@ using namespace tc;
 constexpr int CH = 64;   // chunk length
 constexpr int D = 128;   // dk = dv
 constexpr int NS = 512;           // SIMT threads (warps 0..15): prep, epilogues, solve
-constexpr int kIssuer = NS / 32;  // warp 16 issues every MMA
-constexpr int NT = NS + 32;       // threads per CTA
+constexpr int kIssuer = NS / 32;       // warp 16 issues every MMA
+constexpr int kProducer = kIssuer + 1;  // warp 17 issues every TMA load of raw chunk rows
+constexpr int NT = NS + 64;             // threads per CTA
 constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
@@ -122,7 +124,12 @@ constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 6
 
 // MB_*: MMA groups done (committed by the issuer warp) and raw rows landed (TMA);
 // RDY_*: operands of an MMA group written (one arrival from the SIMT warps).
-enum { MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX, RDY_G, RDY_2B, RDY_2A, RDY_3, RDY_45, kNumMbar };
+// RDY_RAWA: the SIMT warps are done with the region that the next log_alpha / v / w rows
+// land in.
+enum {
+    MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX,
+    RDY_G, RDY_2B, RDY_2A, RDY_3, RDY_45, RDY_RAWA, kNumMbar
+};
 static_assert(kNumMbar <= 16, "mbarrier slots");
 
 // Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
@@ -253,9 +260,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             tma_load_3d(sbase + OFF_RAW_B + x * 8192, &maps.b, 64 * x, h, ts, mbar(MB_RAWB));
         }
     };
-    if (tid == 0) {
-        issue_raw_a(t0);
-        issue_raw_b(t0);
+    if (warp == kProducer) {
+        // One thread of the producer warp stages every chunk's raw rows: q, k, b as soon as
+        // the Sref MMAs of the previous chunk have read the tiles they land on, log_alpha,
+        // v, w once the previous chunk's X [B;P]^T MMAs and its UT solve are done with theirs.
+        if (lane == 0) {
+            issue_raw_a(t0);
+            issue_raw_b(t0);
+            for (int ci = 0; ci + 1 < nchunks; ++ci) {
+                const uint32_t par = (uint32_t)(ci & 1);
+                const int ts = t0 + (ci + 1) * CH;
+                if (!mbar_wait(mbar(MB_2A), par, kWaitNs)) { fault = true; break; }
+                issue_raw_b(ts);
+                if (!mbar_wait(mbar(MB_2B), par, kWaitNs) || !mbar_wait(mbar(RDY_RAWA), par, kWaitNs)) {
+                    fault = true;
+                    break;
+                }
+                issue_raw_a(ts);
+            }
+        }
+        __syncwarp();
     }
 
     if (warp == kIssuer) {
@@ -357,7 +381,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         __syncwarp();
     }
-    const int simt_chunks = warp == kIssuer ? 0 : nchunks;
+    const int simt_chunks = warp < kIssuer ? nchunks : 0;
 
     for (int ci = 0; ci < simt_chunks; ++ci) {
         const int tc0 = t0 + ci * CH;
@@ -582,16 +606,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // ------------------------------------------------------------ 6. D1 += Sref^T [Kh;Qh]^T
         if (tid == 0) mbar_arrive(mbar(RDY_2A));
         // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
-        // The next chunk's q, k, b may land over Kh / Qh / Ql as soon as the Sref MMAs are
-        // done; thread 0 checks between the solve's levels and issues them then.
-        bool raw_b_issued = !(ci + 1 < nchunks);
-        auto try_issue_raw_b = [&]() {
-            if (tid == 0 && !raw_b_issued && mbar_test(mbar(MB_2A), par)) {
-                tc_fence_after();
-                issue_raw_b(tc0 + CH);
-                raw_b_issued = true;
-            }
-        };
         // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
         // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
         // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
@@ -618,7 +632,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         bar_sync_1<NS>();
-        try_issue_raw_b();
         {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 1 per thread)
             const int blk = tid >> 8, base = 32 * blk, r = (tid >> 4) & 15, c = tid & 15;
             const float* a0 = WA + (base + 16 + r) * WS + base;
@@ -650,7 +663,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             WT[(base + 16 + r) * WS + base + c] = -t;
         }
         bar_sync_1<NS>();
-        try_issue_raw_b();
         {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 2 outputs per thread)
             const int c = tid & 31, r0 = tid >> 5;
             float m[2] = {0.f, 0.f};
@@ -694,15 +706,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         fence_proxy_async_smem();
         tc_fence_before();
         bar_sync_1<NS>();
+        if (tid == 0) mbar_arrive(mbar(RDY_RAWA));  // the solve's workspace is dead
 
         fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
         if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
-        if (tid == 0 && ci + 1 < nchunks) {
-            issue_raw_a(tc0 + CH);                   // B / P and the solve's workspace are dead
-            if (!raw_b_issued) issue_raw_b(tc0 + CH);  // Kh / Qh / Ql are dead
-        }
 
         // ------------------------------------------------------------ 7. Y^T as a bf16 A operand
         // Thread (lane L, quarter cp) takes tokens 16cp .. 16cp + 15 (fp32 columns), packed
@@ -776,7 +785,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     // the staged o tile must be read out before shared memory is released or rewritten
     if (tid == 0) bulk_wait_read0();
 
-    if (!fault && p.S_T && warp != kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
+    if (!fault && p.S_T && warp < kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
         tc_fence_after();
         const int cb = 32 * cp;
@@ -788,7 +797,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             p.S_T[soff + (size_t)c * D + L] = u[e] * expf(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
         }
     }
-    if (fault && (tid == 0 || tid == NS)) atomicOr(&g_tc_fault, 1u);
+    if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_tc_fault, 1u);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
