@@ -35,10 +35,11 @@
 //   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
 //             written while they run
-//   3 Gram epilogue + fp32 blocked triangular solve for T (16 -> 32 -> 64)
-//   4 MMA     D1 = X^T [B;P]^T (+ P cross terms)
+//   3 Gram epilogue (B, A, Qm) + fp32 blocked triangular solve for T (16 -> 32 -> 64);
+//     then the P block (after its cross terms) and MMA O^T += X^T P^T (hi / lo)
+//   4 MMA     Y^T = X^T B^T
 //   5 state epilogue: U <- f (.) U, Sref^T (bf16) into tensor memory
-//   6 MMA     D1 += Sref^T [Kh;Qh]^T (+ Qh lo term), then U += X^T Kb (no state read)
+//   6 MMA     Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (+ Qh lo term), then U += X^T Kb
 //   7 Y^T (bf16, tensor memory)  8 MMA R^T = Y^T T^T  9 -R^T (bf16, tensor memory)
 //   10 MMA: O^T -= R^T Qm^T, U -= R^T Eb
 // Sref^T, Y^T and -R^T are A operands read from tensor memory; the others come from shared
@@ -81,7 +82,7 @@ constexpr uint32_t OFF_XL = 7 * kTile;   // X lo
 // row r sits at chunk c ^ (r % 8), so the prep's reads (8 rows, same columns) hit distinct
 // banks. A bf16 [64][128] tile is 2 boxes (8 KB each), an fp32 one 4 boxes.
 //   group A: log_alpha, v, w -> the reused region, free once the previous chunk's
-//            X [B;P]^T MMAs are done;
+//            X^T P^T MMAs are done;
 //   group B: q, k, b         -> over Kh / Qh / Ql, free once its state read is done.
 constexpr uint32_t OFF_RAW_Q = 0;            // bf16, 16 KB each
 constexpr uint32_t OFF_RAW_K = 1 * kTile;
@@ -95,8 +96,8 @@ constexpr uint32_t kSmall = CH * CH * 2;  // 8192
 constexpr uint32_t OFF_QM = 8 * kTile;     // Qm
 constexpr uint32_t OFF_T = OFF_QM + kSmall;  // T, K-major [i][j]: (j/8)*1024 + (i/8)*128 + (i%8)*16 + (j%8)*2
 constexpr uint32_t OFF_REG = OFF_T + kSmall;  // 64 KB reused by phases 3 / 5-6 / 7-10
-constexpr uint32_t OFF_B = OFF_REG;             // B   } [B; P hi] is one 128-row operand
-constexpr uint32_t OFF_PH = OFF_REG + kSmall;   // P hi}
+constexpr uint32_t OFF_B = OFF_REG;             // B
+constexpr uint32_t OFF_PH = OFF_REG + kSmall;   // P hi
 constexpr uint32_t OFF_PL = OFF_REG + 2 * kSmall;
 constexpr int WS = 68;                                // fp32 row stride (16-byte aligned rows)
 constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][WS]
@@ -127,8 +128,8 @@ constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 6
 // RDY_RAWA: the SIMT warps are done with the region that the next log_alpha / v / w rows
 // land in.
 enum {
-    MB_G = 0, MB_2B, MB_2A, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX,
-    RDY_G, RDY_2B, RDY_2A, RDY_3, RDY_45, RDY_RAWA, kNumMbar
+    MB_G = 0, MB_2B, MB_2A, MB_2P, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX,
+    RDY_G, RDY_2B, RDY_2A, RDY_2P, RDY_3, RDY_45, RDY_RAWA, kNumMbar
 };
 static_assert(kNumMbar <= 16, "mbarrier slots");
 
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     if (warp == kProducer) {
         // One thread of the producer warp stages every chunk's raw rows: q, k, b as soon as
         // the Sref MMAs of the previous chunk have read the tiles they land on, log_alpha,
-        // v, w once the previous chunk's X [B;P]^T MMAs and its UT solve are done with theirs.
+        // v, w once the previous chunk's X^T P^T MMAs and its UT solve are done with theirs.
         if (lane == 0) {
             issue_raw_a(t0);
             issue_raw_b(t0);
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 const int ts = t0 + (ci + 1) * CH;
                 if (!mbar_wait(mbar(MB_2A), par, kWaitNs)) { fault = true; break; }
                 issue_raw_b(ts);
-                if (!mbar_wait(mbar(MB_2B), par, kWaitNs) || !mbar_wait(mbar(RDY_RAWA), par, kWaitNs)) {
+                if (!mbar_wait(mbar(MB_2P), par, kWaitNs) || !mbar_wait(mbar(RDY_RAWA), par, kWaitNs)) {
                     fault = true;
                     break;
                 }
@@ -319,28 +320,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
                 if (!mbar_wait(mbar(RDY_2B), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
-                {  // D1 = X^T [B; P]^T
-                    const uint32_t id128 = idesc_bf16(128, 128, true, true);
+                {  // Y^T = X^T B^T
                     const uint32_t id64 = idesc_bf16(128, 64, true, true);
 #pragma unroll
-                    for (int ks = 0; ks < CH / 16; ++ks) {
-                        const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
-                        const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
-                        mma_bf16(tmem + TM_D1, xh, sdesc(sbase + OFF_B + ks * 256, 128, 1024), id128, ks > 0);
-                        mma_bf16(tmem + TM_D1 + 64, xl, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
-                        mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PL + ks * 256, 128, 1024), id64, 1u);
-                    }
+                    for (int ks = 0; ks < CH / 16; ++ks)
+                        mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_XH + ks * 4096, 2048, 128),
+                                 sdesc(sbase + OFF_B + ks * 256, 128, 1024), id64, ks > 0);
                     mma_commit(mbar(MB_2B));
                 }
                 if (!mbar_wait(mbar(RDY_2A), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
-                {  // D1 += Sref^T [Kh; Qh]^T; then U += X^T Kb, which needs no state read
-                    const uint32_t id128 = idesc_bf16(128, 128, false, false);
+                {  // Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T; then U += X^T Kb (no state read)
                     const uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t a = tmem + TM_S + ks * 8;
-                        mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id128, 1u);
+                        mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id64, 1u);
+                        mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QH + ks * 256, 128, 2048), id64, ks > 0);
                         mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
                     }
                     mma_commit(mbar(MB_2A));
@@ -353,6 +349,20 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
                         mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
                     }
+                }
+                if (!mbar_wait(mbar(RDY_2P), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // O^T += X^T P^T (hi / lo)
+                    const uint32_t id64 = idesc_bf16(128, 64, true, true);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks) {
+                        const uint64_t xh = sdesc(sbase + OFF_XH + ks * 4096, 2048, 128);
+                        const uint64_t xl = sdesc(sbase + OFF_XL + ks * 4096, 2048, 128);
+                        mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
+                        mma_bf16(tmem + TM_D1 + 64, xl, sdesc(sbase + OFF_PH + ks * 256, 128, 1024), id64, 1u);
+                        mma_bf16(tmem + TM_D1 + 64, xh, sdesc(sbase + OFF_PL + ks * 256, 128, 1024), id64, 1u);
+                    }
+                    mma_commit(mbar(MB_2P));
                 }
                 if (!mbar_wait(mbar(RDY_3), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
@@ -518,11 +528,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // Thread (lane L, quarter cp) takes Gram columns 32cp .. 32cp + 31: lanes 0..63 are
         // Kb rows (B, then P), lanes 64..127 Eb rows (A, then Qm); column i, row j = L % 64.
         {
-            // lanes 0..63 of the P block: the cross terms still update it
-            if (cp >= 2 && L < 64) {
-                if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
-                tc_fence_after();
-            }
+            // (lanes 0..63 of the P block, which the cross terms still update, are read after
+            // the UT solve)
             float v[32];
             tmem_ld32_wait(tmem + lane_bits + TM_G + 32 * cp, v);
             const int j = L & 63;
@@ -535,21 +542,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     for (int e = 0; e < 8; ++e) f[e] = (ib + 8 * q + e > j) ? v[8 * q + e] : 0.f;
                     store8_bf16(smem, OFF_B + (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16, f);
                 }
-            } else if (L < 64) {  // P_ij, j <= i, split hi / lo (after the cross terms)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float x[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) x[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
-                    uint4 hi, lo;
-                    split2(x[0], x[1], hi.x, lo.x);
-                    split2(x[2], x[3], hi.y, lo.y);
-                    split2(x[4], x[5], hi.z, lo.z);
-                    split2(x[6], x[7], hi.w, lo.w);
-                    const uint32_t o = (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16;
-                    *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
-                    *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
-                }
+            } else if (L < 64) {
+                // P: after the UT solve
             } else if (cp < 2) {  // A_ij, j < i, fp32 for the solve
 #pragma unroll
                 for (int e = 0; e < 32; ++e) WA[(ib + e) * WS + j] = (ib + e > j) ? v[e] : 0.f;
@@ -567,7 +561,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_before();
         if (bar_or_1<NS>(fault)) { fault = true; break; }
 
-        // ------------------------------------------------------------ 4. D1 = X^T [B;P]^T
+        // ------------------------------------------------------------ 4. Y^T = X^T B^T
         if (tid == 0) mbar_arrive(mbar(RDY_2B));
         // ------------------------------------------------------------ 5. state epilogue
         // Thread (lane L, quarter cp) takes key channels 32cp .. 32cp + 31.
@@ -603,7 +597,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_before();
         bar_sync_1<NS>();
 
-        // ------------------------------------------------------------ 6. D1 += Sref^T [Kh;Qh]^T
+        // ------------------------------------------------------------ 6. Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T
         if (tid == 0) mbar_arrive(mbar(RDY_2A));
         // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
         // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
@@ -703,10 +697,38 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const int i = tid & 63, jg = tid >> 6;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
         }
+        // ------------------------------------------------------------ 3c. P block of the Gram
+        // P_ij (j <= i; lanes j = 0..63, columns 64 + i), split hi / lo. The cross terms that
+        // complete it ran behind the main Gram MMAs; its own MMAs (O^T += X^T P^T) only have
+        // to finish before the o epilogue.
+        if (L < 64 && cp >= 2) {
+            if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
+            tc_fence_after();
+            float v[32];
+            tmem_ld32_wait(tmem + lane_bits + TM_G + 32 * cp, v);
+            const int j = L, ib = 32 * (cp & 1);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float x[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
+                uint4 hi, lo;
+                split2(x[0], x[1], hi.x, lo.x);
+                split2(x[2], x[3], hi.y, lo.y);
+                split2(x[4], x[5], hi.z, lo.z);
+                split2(x[6], x[7], hi.w, lo.w);
+                const uint32_t o = (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16;
+                *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
+                *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
+            }
+        }
         fence_proxy_async_smem();
         tc_fence_before();
         bar_sync_1<NS>();
-        if (tid == 0) mbar_arrive(mbar(RDY_RAWA));  // the solve's workspace is dead
+        if (tid == 0) {
+            mbar_arrive(mbar(RDY_2P));
+            mbar_arrive(mbar(RDY_RAWA));  // the solve's workspace is dead
+        }
 
         fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
