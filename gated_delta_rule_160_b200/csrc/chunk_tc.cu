@@ -36,7 +36,8 @@
 //   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
 //             written while they run
 //   3 Gram epilogue (B, A, Qm) + fp32 blocked triangular solve for T (16 -> 32 -> 64);
-//     then the P block (after its cross terms) and MMA O^T += X^T P^T (hi / lo)
+//     the P block (after its cross terms) beside the solve's first level, then MMA
+//     O^T += X^T P^T (hi / lo)
 //   4 MMA     Y^T = X^T B^T
 //   5 state epilogue: U <- f (.) U, Sref^T (bf16) into tensor memory
 //   6 MMA     Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (+ Qh lo term), then U += X^T Kb
@@ -604,10 +605,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
         // and of 32 into 64 with T_21 = -T_22 (A_21 T_11). Rows of A and T are read as float4
         // (the same row for many lanes: broadcast), columns as consecutive floats.
-        if (tid < 64) {
+        // Level 1 runs on warps 2 and 3 (schedulers 2 and 3), so that the P block, whose
+        // tensor-memory lanes only warps on schedulers 0 and 1 can read, is written beside it.
+        if (tid >= 64 && tid < 128) {
             // column jj of block bI, right-looking: once x_l is final, every later row takes
             // its term, so the chain from one row to the next is a single FMA
-            const int bI = tid >> 4, jj = tid & 15, col = 16 * bI + jj;
+            const int bI = (tid - 64) >> 4, jj = tid & 15, col = 16 * bI + jj;
             const float* ablk = WA + 16 * bI * WS + 16 * bI;
             float x[16];
 #pragma unroll
@@ -620,12 +623,40 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 for (int r = l + 1; r < 16; ++r) x[r] = fmaf(-ablk[r * WS + l], x[l], x[r]);
             }
         } else {
-            for (int idx = tid - 64; idx < 64 * 64; idx += NS - 64) {
+            for (int idx = tid < 64 ? tid : tid - 64; idx < 64 * 64; idx += NS - 64) {
                 const int r = idx >> 6, c = idx & 63;
                 if ((c >> 4) > (r >> 4)) WT[r * WS + c] = 0.f;
             }
+            // ---------------------------------------------------------- 3c. P block of the Gram
+            // P_ij (j <= i; lanes j = 0..63, columns 64 + i), split hi / lo, beside level 1.
+            // The cross terms that complete it ran behind the main Gram MMAs; its own MMAs
+            // (O^T += X^T P^T) run during the rest of the solve.
+            if (L < 64 && cp >= 2) {
+                if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
+                tc_fence_after();
+                float v[32];
+                tmem_ld32_wait(tmem + lane_bits + TM_G + 32 * cp, v);
+                const int j = L, ib = 32 * (cp & 1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
+                    uint4 hi, lo;
+                    split2(x[0], x[1], hi.x, lo.x);
+                    split2(x[2], x[3], hi.y, lo.y);
+                    split2(x[4], x[5], hi.z, lo.z);
+                    split2(x[6], x[7], hi.w, lo.w);
+                    const uint32_t o = (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16;
+                    *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
+                    *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+            }
         }
         bar_sync_1<NS>();
+        if (tid == 0) mbar_arrive(mbar(RDY_2P));
         {   // level 2, step 1: M = A_10 T_00 for the two 32-blocks (512 outputs, 1 per thread)
             const int blk = tid >> 8, base = 32 * blk, r = (tid >> 4) & 15, c = tid & 15;
             const float* a0 = WA + (base + 16 + r) * WS + base;
@@ -697,38 +728,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             const int i = tid & 63, jg = tid >> 6;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
         }
-        // ------------------------------------------------------------ 3c. P block of the Gram
-        // P_ij (j <= i; lanes j = 0..63, columns 64 + i), split hi / lo. The cross terms that
-        // complete it ran behind the main Gram MMAs; its own MMAs (O^T += X^T P^T) only have
-        // to finish before the o epilogue.
-        if (L < 64 && cp >= 2) {
-            if (!mbar_wait(mbar(MB_GX), par, kWaitNs)) fault = true;
-            tc_fence_after();
-            float v[32];
-            tmem_ld32_wait(tmem + lane_bits + TM_G + 32 * cp, v);
-            const int j = L, ib = 32 * (cp & 1);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float x[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) x[e] = (ib + 8 * q + e >= j) ? v[8 * q + e] : 0.f;
-                uint4 hi, lo;
-                split2(x[0], x[1], hi.x, lo.x);
-                split2(x[2], x[3], hi.y, lo.y);
-                split2(x[4], x[5], hi.z, lo.z);
-                split2(x[6], x[7], hi.w, lo.w);
-                const uint32_t o = (ib / 8 + q) * 1024 + (j >> 3) * 128 + (j & 7) * 16;
-                *reinterpret_cast<uint4*>(smem + OFF_PH + o) = hi;
-                *reinterpret_cast<uint4*>(smem + OFF_PL + o) = lo;
-            }
-        }
         fence_proxy_async_smem();
         tc_fence_before();
         bar_sync_1<NS>();
-        if (tid == 0) {
-            mbar_arrive(mbar(RDY_2P));
-            mbar_arrive(mbar(RDY_RAWA));  // the solve's workspace is dead
-        }
+        if (tid == 0) mbar_arrive(mbar(RDY_RAWA));  // the solve's workspace is dead
 
         fault |= !mbar_wait(mbar(MB_2B), par, kWaitNs);
         fault |= !mbar_wait(mbar(MB_2A), par, kWaitNs);
