@@ -65,6 +65,7 @@ constexpr int kIssuer = NS / 32;       // warp 16 issues every MMA
 constexpr int kProducer = kIssuer + 1;  // warp 17 issues every TMA load of raw chunk rows
 constexpr int NT = NS + 64;             // threads per CTA
 constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
+constexpr float kLog2e = 1.4426950408889634f;  // cumulative log-decays are kept in base 2
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
 // row groups outermost (LBO = 128 B, SBO = 2048 B): element (row r, channel c) at
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const int cp = tid >> 7;   // column quarter (SIMT threads)
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
-    float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast
+    float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast (base 2)
     float* fscal = scal + 512;                                  // [128] state frame factors
     float* qtot = scal + 640;  // [4][128] sums of log_alpha over tokens 16q .. 16q + 15
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
@@ -404,9 +405,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         {
             // group A: log_alpha, v, w (tokens past the sequence end count as zero); v and w
             // are read after the Gram MMAs are under way.
-            // Cumulative log-decay G, in place over the staged log_alpha rows: thread
-            // (channel c, quarter cp) sums tokens 16cp .. 16cp + 15 of channel c. The totals
-            // of the earlier quarters are added where G is read.
+            // Cumulative log-decay G, in base 2 (G log2(e)), in place over the staged
+            // log_alpha rows: thread (channel c, quarter cp) sums tokens 16cp .. 16cp + 15 of
+            // channel c. The totals of the earlier quarters are added where G is read.
             fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
             {
                 const int c = L;
@@ -415,7 +416,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 for (int r = 0; r < 16; ++r) {
                     const int i = 16 * cp + r;
                     float* gp = reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c));
-                    acc += i < nvalid ? *gp : 0.f;
+                    acc = fmaf(i < nvalid ? *gp : 0.f, kLog2e, acc);
                     *gp = acc;
                 }
                 qtot[128 * cp + c] = acc;
@@ -427,7 +428,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
                 // factor taking the state from the previous chunk's reference frame (or S0)
                 // into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
-                fscal[c] = ci == 0 ? expf(gref) : expf(scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref);
+                fscal[c] = exp2f(ci == 0 ? gref : scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref);
                 scal[buf * 128 + c] = gref;
                 scal[256 + buf * 128 + c] = glast;
             }
@@ -474,15 +475,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 float kh[4], qv[4], kb[4], eb[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    // fast exponential: relative error a few 1e-6 for |arguments| up to ~45,
-                    // well below the 2^-16 carried by the hi/lo operand splits
-                    const float d = gv[e] + (pss < 2 ? dlo[e] : dhi[e]);  // G - Gref
-                    const float ge = __expf(d);
-                    const float gi = __expf(-d);
+                    // (G - Gref) log2(e); the special-function unit's 2^x is far more accurate
+                    // than the 2^-16 carried by the hi/lo operand splits
+                    const float d = gv[e] + (pss < 2 ? dlo[e] : dhi[e]);
+                    const float ge = ex2_approx(d);
+                    const float gi = ex2_approx(-d);
                     kh[e] = kf[e] * ge;
                     qv[e] = qf[e] * ge;
                     kb[e] = kf[e] * gi;
-                    eb[e] = bf[e] * kf[e] * gi;
+                    eb[e] = bf[e] * kb[e];
                 }
                 uint2 qh, ql, kbh, kbl;
                 split2(qv[0], qv[1], qh.x, ql.x);
@@ -819,7 +820,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
             const int c = cb + e;
-            p.S_T[soff + (size_t)c * D + L] = u[e] * expf(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
+            p.S_T[soff + (size_t)c * D + L] = u[e] * exp2f(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
         }
     }
     if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_tc_fault, 1u);

@@ -96,6 +96,14 @@ __device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
     return v;
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32, relative error about 2^-22;
+// subnormal results flush to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // One arrival (release semantics at CTA scope) on an mbarrier.
 __device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
