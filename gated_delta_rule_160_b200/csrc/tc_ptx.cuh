@@ -73,18 +73,27 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+// Has the phase with the given parity completed? If not yet, the thread may sleep until it
+// does, for at most about suspend_ns.
+__device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        "selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity), "r"(suspend_ns)
+        : "memory");
+    return ok != 0;
+}
 // Wait for the phase with the given parity to complete; gives up after timeout_ns.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, uint64_t timeout_ns) {
+    // a thread that finds the phase incomplete sleeps until it completes (or the hint runs
+    // out), instead of spinning on issue slots that other warps of its scheduler need
+    constexpr uint32_t kSuspendNs = 20000;
+    if (mbar_try(mbar, parity, 0u)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        uint32_t ok;
-        asm volatile(
-            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-            "selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(ok)
-            : "r"(mbar), "r"(parity)
-            : "memory");
-        if (ok) return true;
+        if (mbar_try(mbar, parity, kSuspendNs)) return true;
         if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
 }
