@@ -89,9 +89,10 @@ constexpr uint32_t OFF_XL = 7 * kTile;   // X lo
 constexpr uint32_t OFF_RAW_Q = 0;            // bf16, 16 KB each
 constexpr uint32_t OFF_RAW_K = 1 * kTile;
 constexpr uint32_t OFF_RAW_B = 2 * kTile;
-// The o tile of a full chunk is staged as fp32 [64 tokens][128 channels] over Kb hi / Eb
-// (free once the state MMAs are done) and written by one TMA store.
-constexpr uint32_t OFF_OST = 3 * kTile;      // fp32, 32 KB
+// The o tile of a full chunk is staged as fp32 [32 tokens][128 channels] halves over Kb hi
+// and Kb lo (free once the U += X^T Kb MMAs are done) and written by two TMA stores.
+constexpr uint32_t OFF_OST0 = OFF_KBH;       // tokens 0..31, fp32, 16 KB
+constexpr uint32_t OFF_OST1 = OFF_KBL;       // tokens 32..63
 // [64][64] bf16 tiles. MN-major B operands B[n=i][k=j] written by the Gram epilogue:
 //   (i/8)*1024 + (j/8)*128 + (j%8)*16 + (i%8)*2     (SBO = 1024, LBO = 128)
 constexpr uint32_t kSmall = CH * CH * 2;  // 8192
@@ -111,7 +112,7 @@ constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
 // float gref[2][128], glast[2][128], f[128], quarter-chunk log-decay totals [4][128]
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 9 * 128 * 4;
-constexpr uint32_t OFF_TSLOT = OFF_MBAR + 16 * 8;
+constexpr uint32_t OFF_TSLOT = OFF_MBAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
 static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -130,16 +131,16 @@ constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 6
 // RDY_RAWA: the SIMT warps are done with the region that the next log_alpha / v / w rows
 // land in.
 enum {
-    MB_G = 0, MB_2B, MB_2A, MB_2P, MB_3, MB_45, MB_RAWA, MB_RAWB, MB_GX,
+    MB_G = 0, MB_2B, MB_2A, MB_2P, MB_3, MB_45O, MB_45, MB_RAWA, MB_RAWB, MB_GX,
     RDY_G, RDY_2B, RDY_2A, RDY_2P, RDY_3, RDY_45, RDY_RAWA, kNumMbar
 };
-static_assert(kNumMbar <= 16, "mbarrier slots");
+static_assert(kNumMbar <= 24, "mbarrier slots");
 
 // Tensor maps of the six per-token inputs: 3-d {channel, head, token}, 128-byte boxes of
 // 64 tokens with the 128-byte swizzle.
 struct RawMaps {
     CUtensorMap la, q, k, b, v, w;
-    CUtensorMap o;  // fp32 output, used for full chunks (box {128, 1, 64}, no swizzle)
+    CUtensorMap o;  // fp32 output, used for full chunks (box {128, 1, 32}, no swizzle)
 };
 
 __device__ unsigned int g_tc_fault = 0;
@@ -378,15 +379,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
                 if (!mbar_wait(mbar(RDY_45), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
-                {  // O^T -= R^T Qm^T;  U -= R^T Eb
+                {  // O^T -= R^T Qm^T (committed on its own: the o epilogue waits for it only);
+                   // U -= R^T Eb
                     const uint32_t id_o = idesc_bf16(128, 64, false, true);
                     const uint32_t id_rx = idesc_bf16(128, 128, false, true);
 #pragma unroll
-                    for (int ks = 0; ks < CH / 16; ++ks) {
-                        const uint32_t rr = tmem + TM_R + ks * 8;
-                        mma_bf16_ts(tmem + TM_D1 + 64, rr, sdesc(sbase + OFF_QM + ks * 256, 128, 1024), id_o, 1u);
-                        mma_bf16_ts(tmem + TM_U, rr, sdesc(sbase + OFF_E + ks * 4096, 2048, 128), id_rx, 1u);
-                    }
+                    for (int ks = 0; ks < CH / 16; ++ks)
+                        mma_bf16_ts(tmem + TM_D1 + 64, tmem + TM_R + ks * 8, sdesc(sbase + OFF_QM + ks * 256, 128, 1024),
+                                    id_o, 1u);
+                    mma_commit(mbar(MB_45O));
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks)
+                        mma_bf16_ts(tmem + TM_U, tmem + TM_R + ks * 8, sdesc(sbase + OFF_E + ks * 4096, 2048, 128),
+                                    id_rx, 1u);
                     mma_commit(mbar(MB_45));
                 }
             }
@@ -422,6 +427,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 qtot[128 * cp + c] = acc;
             }
             bar_sync_1<NS>();
+            // the previous (full) chunk's o tile, staged before this barrier
+            if (kTmaStoreO<TO> && ci > 0 && tid == 0) {
+                tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tc0 - CH);
+                tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tc0 - CH / 2);
+                bulk_commit();
+            }
             if (tid < D) {
                 const int c = tid;
                 const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
@@ -445,7 +456,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
                 bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
             }
+            // the tiles below overwrite the staged o tile (over Kb hi / lo) and Eb, which the
+            // previous chunk's U -= R^T Eb MMAs read
             if (tid == 0) bulk_wait_read0();
+            if (ci > 0) fault |= !mbar_wait(mbar(MB_45), par ^ 1u, kWaitNs);
             if (bar_or_1<NS>(fault)) {
                 fault = true;
                 break;
@@ -777,7 +791,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 10. output and state MMAs
         if (tid == 0) mbar_arrive(mbar(RDY_45));
-        fault |= !mbar_wait(mbar(MB_45), par, kWaitNs);
+        fault |= !mbar_wait(mbar(MB_45O), par, kWaitNs);
         if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
 
@@ -787,16 +801,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             float ov[16];
             tmem_ld16_wait(tmem + lane_bits + TM_D1 + 64 + 16 * cp, ov);
             if (kTmaStoreO<TO> && nvalid == CH) {
-                // stage the fp32 tile [token][channel] and let one TMA store write it
-                float* ost = reinterpret_cast<float*>(smem + OFF_OST);
+                // stage the fp32 tile [token][channel] in two halves over Kb hi / lo (free:
+                // the U += X^T Kb MMAs ran before the ones just waited for; Eb, which the
+                // U -= R^T Eb MMAs may still read, is untouched); TMA stores write them after
+                // the next barrier (the next chunk's scan, or the one after the loop)
+                float* ost = reinterpret_cast<float*>(smem + (cp < 2 ? OFF_OST0 : OFF_OST1));
 #pragma unroll
-                for (int e = 0; e < 16; ++e) ost[(16 * cp + e) * D + L] = ov[e];
+                for (int e = 0; e < 16; ++e) ost[(16 * (cp & 1) + e) * D + L] = ov[e];
                 fence_proxy_async_smem();
-                bar_sync_1<NS>();
-                if (tid == 0) {
-                    tma_store_3d(&maps.o, sbase + OFF_OST, 0, h, tc0);
-                    bulk_commit();
-                }
             } else {
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -806,10 +818,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         tc_fence_before();
-        bar_sync_1<NS>();
     }
-    // the staged o tile must be read out before shared memory is released or rewritten
-    if (tid == 0) bulk_wait_read0();
+    if (warp < kIssuer) {
+        bar_sync_1<NS>();
+        const int tcl = t0 + (nchunks - 1) * CH;
+        if (kTmaStoreO<TO> && !fault && t1 - tcl == CH && tid == 0) {  // the last chunk's staged o
+            tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tcl);
+            tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tcl + CH / 2);
+            bulk_commit();
+        }
+        // the staged o tile must be read out before shared memory is released or rewritten
+        if (tid == 0) bulk_wait_read0();
+        if (!fault) fault = !mbar_wait(mbar(MB_45), (uint32_t)((nchunks - 1) & 1), kWaitNs);
+    }
 
     if (!fault && p.S_T && warp < kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
@@ -841,14 +862,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Rows of one head of a [T, heads, 128] tensor, in boxes of 64 tokens. swizzled: boxes of
-// 128 bytes per row (64 bf16 / 32 fp32 channels) with the 128-byte swizzle; else whole rows.
+// Rows of one head of a [T, heads, 128] tensor, in boxes of box_rows tokens. swizzled:
+// boxes of 128 bytes per row (64 bf16 / 32 fp32 channels) with the 128-byte swizzle; else
+// whole rows.
 bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap* m, const void* base, bool fp32, int heads,
-                 int T, bool swizzled) {
+                 int T, bool swizzled, int box_rows = CH) {
     const cuuint64_t es = fp32 ? 4 : 2;
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)T};
     cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)heads * D * es};
-    cuuint32_t box[3] = {swizzled ? (cuuint32_t)(128 / es) : (cuuint32_t)D, 1u, (cuuint32_t)CH};
+    cuuint32_t box[3] = {swizzled ? (cuuint32_t)(128 / es) : (cuuint32_t)D, 1u, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -869,7 +891,7 @@ cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
         !encode_rows(fn, &maps.w, p.w, false, p.h_v, p.T_total, true))
         return cudaErrorInvalidValue;
     if (sizeof(TO) == 4) {
-        if (!encode_rows(fn, &maps.o, p.o, true, p.h_v, p.T_total, false)) return cudaErrorInvalidValue;
+        if (!encode_rows(fn, &maps.o, p.o, true, p.h_v, p.T_total, false, CH / 2)) return cudaErrorInvalidValue;
     } else {
         maps.o = maps.la;  // unused: bf16 outputs take plain stores
     }
