@@ -19,10 +19,10 @@
 // Precision: bf16 operands round to 8 significant bits, and the outputs of this
 // recurrence have max|o| / rms(o) of 10 to 15, so one rounding on a dominant term costs
 // more than the 2e-2 * rms(o) error budget. The terms that carry the output and the
-// state -- P (query/key Gram block), P X and Kb^T X -- are therefore computed with both
-// operands split into bf16 hi + lo parts (three MMAs: hi*hi + lo*hi + hi*lo, about 16
-// significant bits); Qh Sref splits Qh only (Qh_hi Sref + Qh_lo Sref); the erase path
-// (A, B, Qm, T, Y, R) stays in plain bf16.
+// state -- P (query/key Gram block), P X, Kb^T X and Qh Sref -- are therefore computed with
+// both operands split into bf16 hi + lo parts (three MMAs: hi*hi + lo*hi + hi*lo, about 16
+// significant bits); the erase path (A, B, Qm, T, Y, R) stays in plain bf16. (Qh Sref
+// carries the whole output when the state dominates it: a long history, a large S0.)
 //
 // Phases per chunk. Sixteen SIMT warps take part in each (thread t serves tensor-memory
 // lane t % 128 and column quarter t / 128): the phases are chains of dependent
@@ -39,8 +39,8 @@
 //     the P block (after its cross terms) beside the solve's first level, then MMA
 //     O^T += X^T P^T (hi / lo)
 //   4 MMA     Y^T = X^T B^T
-//   5 state epilogue: U <- f (.) U, Sref^T (bf16) into tensor memory
-//   6 MMA     Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (+ Qh lo term), then U += X^T Kb
+//   5 state epilogue: U <- f (.) U, Sref^T (bf16 hi / lo) into tensor memory
+//   6 MMA     Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (hi / lo), then U += X^T Kb
 //   7 Y^T (bf16, tensor memory)  8 MMA R^T = Y^T T^T  9 -R^T (bf16, tensor memory)
 //   10 MMA: O^T -= R^T Qm^T, U -= R^T Eb
 // Sref^T, Y^T and -R^T are A operands read from tensor memory; the others come from shared
@@ -109,9 +109,10 @@ constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
 constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
 constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
-// float gref[2][128], glast[2][128], f[128], quarter-chunk log-decay totals [4][128]
+// float gref[2][128], glast[2][128], frame factors f[2][128], quarter-chunk log-decay
+// totals [4][128]
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
-constexpr uint32_t OFF_MBAR = OFF_SCAL + 9 * 128 * 4;
+constexpr uint32_t OFF_MBAR = OFF_SCAL + 10 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 24 * 8;
 constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
 static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
@@ -122,7 +123,10 @@ constexpr uint32_t TM_G = 0;     // Gram (transposed): lanes [Kb j ; Eb j], cols
 constexpr uint32_t TM_D1 = 128;  // [Y^T | O^T]
 constexpr uint32_t TM_R = 256;   // R^T
 constexpr uint32_t TM_U = 384;   // state, lanes m (value channel), cols c (key channel)
-constexpr uint32_t TM_S = 320;   // Sref^T as a bf16 A operand (packed pairs), 64 columns
+constexpr uint32_t TM_S = 320;   // Sref^T hi as a bf16 A operand (packed pairs), 64 columns
+// Sref^T lo, over the B / A blocks of the Gram (read by its epilogue before the state
+// epilogue writes this; the next Gram comes after the Sref MMAs are done)
+constexpr uint32_t TM_SL = TM_G;
 // Y^T and -R^T also serve as bf16 A operands from tensor memory, packed over the first 32
 // columns of their own fp32 accumulators (TM_D1, TM_R).
 
@@ -201,8 +205,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const uint32_t sbase = smem_u32(smem);
     const uint32_t lane_bits = (uint32_t)(L & 96) << 16;
     float* scal = reinterpret_cast<float*>(smem + OFF_SCAL);  // [0..255] gref, [256..511] glast (base 2)
-    float* fscal = scal + 512;                                  // [128] state frame factors
-    float* qtot = scal + 640;  // [4][128] sums of log_alpha over tokens 16q .. 16q + 15
+    float* fscal = scal + 512;  // [2][128] state frame factors (applied one after the other)
+    float* qtot = scal + 768;  // [4][128] sums of log_alpha over tokens 16q .. 16q + 15
     float* WA = reinterpret_cast<float*>(smem + OFF_WA);
     float* WT = reinterpret_cast<float*>(smem + OFF_WT);
     float* WM = reinterpret_cast<float*>(smem + OFF_WM);
@@ -333,14 +337,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 }
                 if (!mbar_wait(mbar(RDY_2A), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
-                {  // Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T; then U += X^T Kb (no state read)
+                {  // Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (hi / lo); then U += X^T Kb (no state read)
                     const uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint32_t a = tmem + TM_S + ks * 8;
+                        const uint32_t a = tmem + TM_S + ks * 8, al = tmem + TM_SL + ks * 8;
+                        const uint64_t qh = sdesc(sbase + OFF_QH + ks * 256, 128, 2048);
                         mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id64, 1u);
-                        mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QH + ks * 256, 128, 2048), id64, ks > 0);
+                        mma_bf16_ts(tmem + TM_D1 + 64, a, qh, id64, ks > 0);
                         mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
+                        mma_bf16_ts(tmem + TM_D1 + 64, al, qh, id64, 1u);
                     }
                     mma_commit(mbar(MB_2A));
                     const uint32_t id_xx = idesc_bf16(128, 128, true, true);
@@ -437,9 +443,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 const int c = tid;
                 const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
                 const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
-                // factor taking the state from the previous chunk's reference frame (or S0)
-                // into this chunk's: exp(G_last' - Gref' + Gref), or exp(Gref)
-                fscal[c] = exp2f(ci == 0 ? gref : scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c] + gref);
+                // factors taking the state from the previous chunk's reference frame into
+                // this chunk's: exp(G_last' - Gref') (to the state itself), then exp(Gref).
+                // Two factors, not their product: with strong decay the product underflows
+                // where the scaled state does not. (S0 takes exp(Gref) alone.)
+                fscal[c] = exp2f(ci == 0 ? gref : scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c]);
+                fscal[128 + c] = exp2f(gref);
                 scal[buf * 128 + c] = gref;
                 scal[256 + buf * 128 + c] = glast;
             }
@@ -593,21 +602,24 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             } else {
                 tmem_ld32_wait(tmem + lane_bits + TM_U + cb, u);
                 const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
+                const float4* g4 = reinterpret_cast<const float4*>(fscal + 128 + cb);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 f = f4[e4];
-                    u[4 * e4] *= f.x;
-                    u[4 * e4 + 1] *= f.y;
-                    u[4 * e4 + 2] *= f.z;
-                    u[4 * e4 + 3] *= f.w;
+                    const float4 f = f4[e4], gg = g4[e4];
+                    u[4 * e4] = u[4 * e4] * f.x * gg.x;
+                    u[4 * e4 + 1] = u[4 * e4 + 1] * f.y * gg.y;
+                    u[4 * e4 + 2] = u[4 * e4 + 2] * f.z * gg.z;
+                    u[4 * e4 + 3] = u[4 * e4 + 3] * f.w * gg.w;
                 }
             }
             tmem_st32(tmem + lane_bits + TM_U + cb, u);
-            // Sref^T as a bf16 A operand: key channels cb .. cb + 31 in columns cb/2 .. +15
-            uint32_t pk[16];
+            // Sref^T as bf16 hi / lo A operands: key channels cb .. cb + 31 in columns
+            // cb/2 .. +15 of TM_S (hi) and TM_SL (lo)
+            uint32_t pk[16], pl[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(u[2 * e], u[2 * e + 1]);
+            for (int e = 0; e < 16; ++e) split2(u[2 * e], u[2 * e + 1], pk[e], pl[e]);
             tmem_st16(tmem + lane_bits + TM_S + 16 * cp, pk);
+            tmem_st16(tmem + lane_bits + TM_SL + 16 * cp, pl);
             tmem_wait_st();
         }
         tc_fence_before();
