@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "prefill_b8_h16_t4096"
 DECODE = "decode_256seq_h32"
+SERVING_TOKENS = 4  # tokens per sequence in one serving-decode step (a verify step)
 DECODE_TIMED_STEPS = 64
 
 
@@ -136,6 +137,15 @@ def prefill_bytes(wl, lengths) -> int:
                  + wl.h_v * (2 * wl.dv * es + wl.dk * es + 4 * wl.dk + 4 * wl.dv))
     state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
     return T * per_token + state * (2 if wl.S0_std else 1)
+
+
+def serving_bytes(wl, n_tok: int) -> int:
+    """Algorithmic bytes of one serving-decode step: each active state read and written
+    once, plus n_tok tokens of input and output per sequence."""
+    es = torch.finfo(wl.dtype).bits // 8
+    n = wl.n_seq
+    io = n * n_tok * (wl.h_qk * 2 * wl.dk * es + wl.h_v * (2 * wl.dv * es + wl.dk * es + 4 * wl.dk + 4 * wl.dv))
+    return io + 2 * n * wl.h_v * wl.dk * wl.dv * 4
 
 
 def decode_bytes(wl) -> int:
@@ -315,6 +325,43 @@ def main():
                            "algorithmic_bytes_per_launch": dbytes}}
     del S, dec_in
 
+    # ---------------- serving decode: states in a slot pool, SERVING_TOKENS per step
+    pool = torch.zeros((2 * dwl.n_seq, dwl.h_v, dwl.dk, dwl.dv), dtype=torch.float32, device=dev)
+    perm = torch.randperm(2 * dwl.n_seq, generator=torch.Generator().manual_seed(dwl.seed))[:dwl.n_seq]
+    pool[perm.to(dev)] = W.decode_state(dwl, dev)
+    slots = perm.to(torch.int32).to(dev)
+    srv_in = []
+    for s_ in range(2):
+        t_ = W.token_inputs(dwl.n_seq * SERVING_TOKENS, dwl.h_qk, dwl.h_v, dwl.dk, dwl.dv, dwl.dtype, dev,
+                            dwl.seed * 7919 + s_)
+        srv_in.append({k: t.view(dwl.n_seq, SERVING_TOKENS, *t.shape[1:]) for k, t in t_.items()})
+    so = torch.empty((dwl.n_seq, SERVING_TOKENS, dwl.h_v, dwl.dv), dtype=torch.float32, device=dev)
+    sstep = lambda i: G.gdn2_decode_multi(*(srv_in[i % 2][k] for k in ("q", "k", "v", "log_alpha", "b", "w")),
+                                          pool, slots=slots, o=so, stream=stream)
+    for i in range(5):
+        sstep(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for i in range(DECODE_TIMED_STEPS):
+        sstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    sms = max_over_ranks(e0.elapsed_time(e1) / DECODE_TIMED_STEPS, world)
+    sbytes = serving_bytes(dwl, SERVING_TOKENS)
+    sach = sbytes / (sms / 1000.0) / 1e9
+    serving = {"metric": "GDN-2 serving decode tokens/s",
+               "value": world * dwl.n_seq * SERVING_TOKENS / (sms / 1000.0), "unit": "tokens/s",
+               "ms_per_step": sms, "steps": DECODE_TIMED_STEPS,
+               "config": {"workload": f"{DECODE}, states at seeded-random slots of a {2 * dwl.n_seq}-state "
+                                      f"pool, {SERVING_TOKENS} tokens per sequence and step",
+                          "n_seq": dwl.n_seq, "heads": dwl.h_v, "n_tok": SERVING_TOKENS,
+                          "pool_slots": 2 * dwl.n_seq},
+               "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s", "frac": sach / hbm,
+                            "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                            "algorithmic_bytes_per_launch": sbytes}}
+    del pool, srv_in, so
+
     # ---------------- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -364,6 +411,7 @@ def main():
                        "l2": "inputs (1.07 GB per rank) larger than L2; no flush"},
             "roofline": roofline,
             "decode": decode,
+            "serving_decode": serving,
             "e2e": e2e,
             "cpu_baseline": base,
             "clocks": clocks.summary(),

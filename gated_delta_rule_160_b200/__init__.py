@@ -19,6 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgdn2.so")
 
 GDN2_F32, GDN2_BF16 = 0, 1
+GDN2_DECODE_MAX_TOKENS = 8  # tokens per sequence in one gdn2_decode_multi call (gdn2.h)
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_CUDA"}
 ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_decode_step",
                  "gdn2_chunk_fwd_noalloc", "gdn2_last_error_string", "gdn2_version")
@@ -56,6 +57,9 @@ def load_library(path: str = LIB_PATH):
     lib.gdn2_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(Shape)] + [vp] * 10 + [vp]
     lib.gdn2_decode_step.restype = ctypes.c_int
     lib.gdn2_decode_step.argtypes = [ctypes.POINTER(Shape)] + [vp] * 9
+    lib.gdn2_decode_multi.restype = ctypes.c_int
+    lib.gdn2_decode_multi.argtypes = ([ctypes.POINTER(Shape), ctypes.c_int] + [vp] * 8
+                                      + [ctypes.c_int, vp, vp, vp])
     lib.gdn2_last_error_string.restype = ctypes.c_char_p
     lib.gdn2_last_error_string.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -156,3 +160,28 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None, out_dtype
     _check(lib.gdn2_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                                 _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream_handle(stream)))
     return o
+
+
+def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_steps=None,
+                      want_steps: bool = False, stream=None, out_dtype=torch.float32):
+    """Serving decode: n_tok new tokens for each of N sequences whose states sit in a pool.
+
+    q,k [N,n_tok,Hqk,dk]; v,w [N,n_tok,Hv,dv]; log_alpha (fp32), b [N,n_tok,Hv,dk];
+    S_pool fp32 [n_slots,Hv,dk,dv], updated in place; slots int32 [N] (slot of each
+    sequence; negative = inactive, skipped) or None (slot n). Returns (o [N,n_tok,Hv,dv],
+    S_steps fp32 [N,n_tok,Hv,dk,dv] -- the state after each token -- or None)."""
+    lib = load_library()
+    if o is not None:
+        out_dtype = o.dtype
+    N, n_tok, h_qk, dk = q.shape
+    _, _, h_v, dv = v.shape
+    shape = Shape(int(N), int(N * n_tok), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v.dtype),
+                  _dtype_code(out_dtype))
+    if o is None:
+        o = torch.empty((N, n_tok, h_v, dv), dtype=out_dtype, device=v.device)
+    if S_steps is None and want_steps:
+        S_steps = torch.empty((N, n_tok, h_v, dk, dv), dtype=torch.float32, device=v.device)
+    _check(lib.gdn2_decode_multi(ctypes.byref(shape), int(n_tok), _ptr(slots), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
+                                 _ptr(o), _ptr(S_steps), _stream_handle(stream)))
+    return o, S_steps

@@ -89,6 +89,7 @@ Params make_params(const gdn2_shape* sh, const void* q, const void* k, const voi
     p.T_fixed = cu ? 0 : sh->T_total / sh->n_seq;
     p.q = q; p.k = k; p.v = v; p.log_alpha = la; p.b = b; p.w = w;
     p.S0 = S0; p.cu_seqlens = cu; p.o = o; p.S_T = S_T; p.order = nullptr;
+    p.n_tok = 1; p.slots = nullptr; p.n_slots = sh->n_seq; p.S_steps = nullptr;
     return p;
 }
 
@@ -168,6 +169,38 @@ gdn2_status gdn2_decode_step(const gdn2_shape* shape, const void* q, const void*
     st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
     if (st != GDN2_OK) return st;
     Params p = make_params(shape, q, k, v, log_alpha, b, w, nullptr, nullptr, o, S);
+    cudaError_t e = launch_decode(p, shape->dtype, shape->o_dtype, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
+gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t* slots, const void* q,
+                              const void* k, const void* v, const float* log_alpha, const void* b, const void* w,
+                              float* S_pool, int n_slots, void* o, float* S_steps, gdn2_stream_t stream) {
+    gdn2_status st = check_shape(shape);
+    if (st != GDN2_OK) return st;
+    if (n_tok < 1 || n_tok > GDN2_DECODE_MAX_TOKENS)
+        return fail(GDN2_ERR_INVALID_ARG, "n_tok = %d outside 1..%d", n_tok, GDN2_DECODE_MAX_TOKENS);
+    if ((long long)shape->n_seq * n_tok != shape->T_total)
+        return fail(GDN2_ERR_INVALID_ARG, "T_total = %d is not n_seq * n_tok = %d * %d", shape->T_total,
+                    shape->n_seq, n_tok);
+    if (n_slots < 1 || (!slots && n_slots < shape->n_seq))
+        return fail(GDN2_ERR_INVALID_ARG, "n_slots = %d too small (n_seq = %d, slots %s)", n_slots, shape->n_seq,
+                    slots ? "given" : "NULL");
+    if ((long long)shape->n_seq * shape->h_v > 0x7fffffffLL || (long long)n_slots * shape->h_v > 0x7fffffffLL)
+        return fail(GDN2_ERR_UNSUPPORTED, "n_seq * h_v or n_slots * h_v too large for one launch");
+    const NamedPtr ps[] = {
+        {"q", q, true}, {"k", k, true}, {"v", v, true}, {"log_alpha", log_alpha, true}, {"b", b, true},
+        {"w", w, true}, {"S_pool", S_pool, true}, {"o", o, true}, {"slots", slots, false},
+        {"S_steps", S_steps, false},
+    };
+    st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
+    if (st != GDN2_OK) return st;
+    Params p = make_params(shape, q, k, v, log_alpha, b, w, nullptr, nullptr, o, S_pool);
+    p.n_tok = n_tok;
+    p.slots = slots;
+    p.n_slots = n_slots;
+    p.S_steps = S_steps;
     cudaError_t e = launch_decode(p, shape->dtype, shape->o_dtype, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
     return ok();

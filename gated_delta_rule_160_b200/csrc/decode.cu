@@ -1,4 +1,5 @@
-// decode.cu -- one decode step: one new token per sequence, state updated in place.
+// decode.cu -- decode steps: n_tok (usually 1) new tokens per sequence, state updated in
+// place (in a slot of a state pool for serving), optionally every intermediate state.
 //
 // The step is bound by HBM: the fp32 state [dk, dv] of every (sequence, value head) is
 // read once and written once; everything else is a few hundred bytes. One CTA of 256
@@ -21,105 +22,135 @@ namespace {
 
 constexpr int kThreads = 256;
 
-template <int DK, int DV, typename T, typename TO>
+// kMulti: several tokens, or every intermediate state, so the state is kept in registers
+// across tokens and stored at the end; otherwise each state row is stored as soon as it is
+// updated, which keeps fewer registers live (two CTAs per SM for dk = dv = 128). All the
+// tokens' inputs are staged in shared memory before the first one is applied, so HBM latency
+// is paid once per step, not once per token.
+template <int DK, int DV, typename T, typename TO, bool kMulti>
 __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     constexpr int TPR = DV / 4;          // threads per state row
     constexpr int RG = kThreads / TPR;   // row groups
     constexpr int RPT = DK / RG;         // rows per thread
-    __shared__ float sa[DK], sk[DK], sq[DK], se[DK], sx[DV];
-    __shared__ float4 red[2][RG][TPR];
-    __shared__ float dots[2];
+    constexpr int NTM = kMulti ? GDN2_DECODE_MAX_TOKENS : 1;
+    __shared__ float sa[NTM][DK], sk[NTM][DK], sq[NTM][DK], se[NTM][DK], sx[NTM][DV];
+    __shared__ float4 red[2][2][RG][TPR];  // [token parity][r | p]
+    __shared__ float dots[NTM][2];
 
     const int item = blockIdx.x;  // n * h_v + h
     const int n = item / p.h_v;
     const int h = item % p.h_v;
     const int g = h / (p.h_v / p.h_qk);
+    const int slot = p.slots ? p.slots[n] : n;
+    if (slot < 0 || slot >= p.n_slots) return;  // an inactive sequence: nothing to do
     const int cg = threadIdx.x % TPR;
     const int rg = threadIdx.x / TPR;
-    float* S = p.S_T + (size_t)item * DK * DV;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int n_tok = kMulti ? p.n_tok : 1;
+    float* S = p.S_T + ((size_t)slot * p.h_v + h) * DK * DV;
 
     float4 s[RPT];
 #pragma unroll
     for (int i = 0; i < RPT; ++i)
         s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(rg + RG * i) * DV) + cg);
 
-    const size_t tq = (size_t)n * p.h_qk + g;  // token n of sequence n
-    const size_t tv = (size_t)n * p.h_v + h;
-    for (int c = threadIdx.x; c < DK; c += kThreads) {
+    // every token's decay, key, query, erase and write vectors
+    for (int idx = threadIdx.x; idx < n_tok * DK; idx += kThreads) {
+        const int t = idx / DK, c = idx % DK;
+        const size_t row = (size_t)n * n_tok + t;
+        const size_t tq = row * p.h_qk + g, tv = row * p.h_v + h;
         const float kv = to_f32(static_cast<const T*>(p.k)[tq * DK + c]);
-        sk[c] = kv;
-        sq[c] = to_f32(static_cast<const T*>(p.q)[tq * DK + c]);
-        sa[c] = expf(p.log_alpha[tv * DK + c]);
-        se[c] = to_f32(static_cast<const T*>(p.b)[tv * DK + c]) * kv;
+        sk[t][c] = kv;
+        sq[t][c] = to_f32(static_cast<const T*>(p.q)[tq * DK + c]);
+        sa[t][c] = expf(p.log_alpha[tv * DK + c]);
+        se[t][c] = to_f32(static_cast<const T*>(p.b)[tv * DK + c]) * kv;
     }
-    for (int c = threadIdx.x; c < DV; c += kThreads)
-        sx[c] = to_f32(static_cast<const T*>(p.w)[tv * DV + c]) *
-                to_f32(static_cast<const T*>(p.v)[tv * DV + c]);
+    for (int idx = threadIdx.x; idx < n_tok * DV; idx += kThreads) {
+        const int t = idx / DV, c = idx % DV;
+        const size_t tv = ((size_t)n * n_tok + t) * p.h_v + h;
+        sx[t][c] = to_f32(static_cast<const T*>(p.w)[tv * DV + c]) * to_f32(static_cast<const T*>(p.v)[tv * DV + c]);
+    }
     __syncthreads();
-    if (threadIdx.x < 32) {
+    // q . (b (.) k) and q . k of every token: warp t takes token t
+    for (int t = warp; t < n_tok; t += kThreads / 32) {
         float d1 = 0.f, d2 = 0.f;
-        for (int c = threadIdx.x; c < DK; c += 32) {
-            d1 += sq[c] * se[c];
-            d2 += sq[c] * sk[c];
+        for (int c = lane; c < DK; c += 32) {
+            d1 += sq[t][c] * se[t][c];
+            d2 += sq[t][c] * sk[t][c];
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             d1 += __shfl_xor_sync(0xffffffffu, d1, off);
             d2 += __shfl_xor_sync(0xffffffffu, d2, off);
         }
-        if (threadIdx.x == 0) {
-            dots[0] = d1;
-            dots[1] = d2;
+        if (lane == 0) {
+            dots[t][0] = d1;
+            dots[t][1] = d2;
         }
     }
 
-    float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r;
+    // the state stays in registers from token to token
+    for (int t = 0; t < n_tok; ++t) {
+        const size_t row = (size_t)n * n_tok + t;  // token t of sequence n
+        const size_t tv = row * p.h_v + h;
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f), pq = r;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int row = rg + RG * i;
-        const float a = sa[row], kv = sk[row], qv = sq[row];
-        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-        r.x = fmaf(kv, s[i].x, r.x); r.y = fmaf(kv, s[i].y, r.y);
-        r.z = fmaf(kv, s[i].z, r.z); r.w = fmaf(kv, s[i].w, r.w);
-        pq.x = fmaf(qv, s[i].x, pq.x); pq.y = fmaf(qv, s[i].y, pq.y);
-        pq.z = fmaf(qv, s[i].z, pq.z); pq.w = fmaf(qv, s[i].w, pq.w);
-    }
-    red[0][rg][cg] = r;
-    red[1][rg][cg] = pq;
-    __syncthreads();
-    r = make_float4(0.f, 0.f, 0.f, 0.f);
-    pq = r;
+        for (int i = 0; i < RPT; ++i) {
+            const int rw = rg + RG * i;
+            const float a = sa[t][rw], kv = sk[t][rw], qv = sq[t][rw];
+            s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+            r.x = fmaf(kv, s[i].x, r.x); r.y = fmaf(kv, s[i].y, r.y);
+            r.z = fmaf(kv, s[i].z, r.z); r.w = fmaf(kv, s[i].w, r.w);
+            pq.x = fmaf(qv, s[i].x, pq.x); pq.y = fmaf(qv, s[i].y, pq.y);
+            pq.z = fmaf(qv, s[i].z, pq.z); pq.w = fmaf(qv, s[i].w, pq.w);
+        }
+        // partial sums in the buffer of this token's parity: the one of the token before is
+        // still being read, the one of two tokens before is free (a barrier lies between)
+        red[t & 1][0][rg][cg] = r;
+        red[t & 1][1][rg][cg] = pq;
+        __syncthreads();
+        r = make_float4(0.f, 0.f, 0.f, 0.f);
+        pq = r;
 #pragma unroll
-    for (int j = 0; j < RG; ++j) {
-        const float4 a = red[0][j][cg], b = red[1][j][cg];
-        r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
-        pq.x += b.x; pq.y += b.y; pq.z += b.z; pq.w += b.w;
-    }
-    const float4 x = *reinterpret_cast<const float4*>(sx + 4 * cg);
+        for (int j = 0; j < RG; ++j) {
+            const float4 a = red[t & 1][0][j][cg], b = red[t & 1][1][j][cg];
+            r.x += a.x; r.y += a.y; r.z += a.z; r.w += a.w;
+            pq.x += b.x; pq.y += b.y; pq.z += b.z; pq.w += b.w;
+        }
+        const float4 x = *reinterpret_cast<const float4*>(&sx[t][4 * cg]);
+        float* Ss = kMulti && p.S_steps ? p.S_steps + (row * p.h_v + h) * DK * DV : nullptr;
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int row = rg + RG * i;
-        const float e = -se[row], kv = sk[row];
-        float4 t = s[i];
-        t.x = fmaf(kv, x.x, fmaf(e, r.x, t.x));
-        t.y = fmaf(kv, x.y, fmaf(e, r.y, t.y));
-        t.z = fmaf(kv, x.z, fmaf(e, r.z, t.z));
-        t.w = fmaf(kv, x.w, fmaf(e, r.w, t.w));
-        __stcs(reinterpret_cast<float4*>(S + (size_t)row * DV) + cg, t);
+        for (int i = 0; i < RPT; ++i) {
+            const int rw = rg + RG * i;
+            const float e = -se[t][rw], kv = sk[t][rw];
+            s[i].x = fmaf(kv, x.x, fmaf(e, r.x, s[i].x));
+            s[i].y = fmaf(kv, x.y, fmaf(e, r.y, s[i].y));
+            s[i].z = fmaf(kv, x.z, fmaf(e, r.z, s[i].z));
+            s[i].w = fmaf(kv, x.w, fmaf(e, r.w, s[i].w));
+            if (!kMulti) __stcs(reinterpret_cast<float4*>(S + (size_t)rw * DV) + cg, s[i]);
+            if (Ss) __stcs(reinterpret_cast<float4*>(Ss + (size_t)rw * DV) + cg, s[i]);
+        }
+        if (rg == 0) {
+            const float qe = dots[t][0], qk = dots[t][1];
+            TO* o = static_cast<TO*>(p.o) + tv * DV + 4 * cg;
+            o[0] = from_f32<TO>(pq.x - qe * r.x + qk * x.x);
+            o[1] = from_f32<TO>(pq.y - qe * r.y + qk * x.y);
+            o[2] = from_f32<TO>(pq.z - qe * r.z + qk * x.z);
+            o[3] = from_f32<TO>(pq.w - qe * r.w + qk * x.w);
+        }
     }
-    if (rg == 0) {
-        const float qe = dots[0], qk = dots[1];
-        TO* o = static_cast<TO*>(p.o) + tv * DV + 4 * cg;
-        o[0] = from_f32<TO>(pq.x - qe * r.x + qk * x.x);
-        o[1] = from_f32<TO>(pq.y - qe * r.y + qk * x.y);
-        o[2] = from_f32<TO>(pq.z - qe * r.z + qk * x.z);
-        o[3] = from_f32<TO>(pq.w - qe * r.w + qk * x.w);
+    if (kMulti) {
+#pragma unroll
+        for (int i = 0; i < RPT; ++i) __stcs(reinterpret_cast<float4*>(S + (size_t)(rg + RG * i) * DV) + cg, s[i]);
     }
 }
 
 template <int DK, int DV, typename T, typename TO>
 cudaError_t launch_dec(const Params& p, cudaStream_t st) {
-    decode_kernel<DK, DV, T, TO><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
+    if (p.n_tok > 1 || p.S_steps)
+        decode_kernel<DK, DV, T, TO, true><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
+    else
+        decode_kernel<DK, DV, T, TO, false><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

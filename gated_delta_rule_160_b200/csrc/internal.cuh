@@ -24,6 +24,11 @@ struct Params {
     void* o;
     float* S_T;                // nullable (decode: the in/out state)
     const int32_t* order;      // nullable: sequences longest first (varlen scheduling)
+    // decode only
+    int n_tok;                 // tokens per sequence and step (1..8)
+    const int32_t* slots;      // nullable: state slot of each sequence in S_T's pool
+    int n_slots;               // states in the pool
+    float* S_steps;            // nullable: state after each token [n_seq, n_tok, h_v, dk, dv]
 };
 
 // Token range [t0, t1) of sequence n.

@@ -118,6 +118,31 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_shape* shape,
                              float* S, void* o, gdn2_stream_t stream);
 
 /*
+ * Serving-style decode: n_tok (1..GDN2_DECODE_MAX_TOKENS) new tokens for each of the n_seq
+ * sequences, whose states live in a pool. The same recurrence as gdn2_decode_step, token
+ * after token; the pages describe single-token decode only, and the slot pool and the
+ * multi-token step are interface choices for continuous batching and for verifying
+ * drafted tokens.
+ *   shape->T_total must equal n_seq * n_tok; token t of sequence n is row n * n_tok + t of
+ *   q, k, v, log_alpha, b, w and o (layouts as above).
+ *   S_pool [n_slots, h_v, dk, dv] float32: sequence n reads and updates, in place, the state
+ *   in slot slots[n] (slots: device int32 [n_seq]; NULL means slot n, and then n_slots must
+ *   be at least n_seq). A sequence whose slot is negative or >= n_slots is skipped: its
+ *   rows of o are not written and no state is touched. Two active sequences must not share
+ *   a slot (they would race).
+ *   S_steps (nullable) [n_seq, n_tok, h_v, dk, dv] float32 receives the state after each
+ *   token, so that a caller that accepts only the first j drafted tokens can put back the
+ *   state after token j - 1 (S_pool itself always ends after all n_tok tokens).
+ * Errors as for the other calls; slot values are only checked on the device (skipped).
+ */
+#define GDN2_DECODE_MAX_TOKENS 8
+GDN2_API gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t* slots,
+                              const void* q, const void* k, const void* v,
+                              const float* log_alpha, const void* b, const void* w,
+                              float* S_pool, int n_slots, void* o, float* S_steps,
+                              gdn2_stream_t stream);
+
+/*
  * Prefill for callers that cannot allocate device memory. The pages have no counterpart:
  * this is an interface choice. It computes exactly what gdn2_chunk_fwd computes (same
  * kernels, same arguments, no workspace), for callers that have no way to give the

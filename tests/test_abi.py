@@ -85,3 +85,18 @@ def test_workspace_size(lib):
 
 def test_version(lib):
     assert lib.gdn2_version() >= 100
+
+
+def test_decode_multi_rejects_before_device_work(lib):
+    import gated_delta_rule_160_b200 as g
+    nul = [None] * 8
+
+    def call(sh, n_tok, n_slots, slots=None):
+        return lib.gdn2_decode_multi(ctypes.byref(sh), n_tok, slots, *nul[:7], n_slots, None, None, None)
+
+    sh = _shape(g, n_seq=4, T_total=12)
+    assert call(sh, 0, 4) == 1 and b"n_tok = 0" in lib.gdn2_last_error_string()
+    assert call(sh, g.GDN2_DECODE_MAX_TOKENS + 1, 4) == 1
+    assert call(sh, 2, 4) == 1 and b"not n_seq * n_tok" in lib.gdn2_last_error_string()
+    assert call(sh, 3, 3) == 1 and b"n_slots = 3 too small" in lib.gdn2_last_error_string()
+    assert call(sh, 3, 4) == 1 and b"q is NULL" in lib.gdn2_last_error_string()
