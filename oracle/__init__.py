@@ -8,6 +8,9 @@ The arithmetic lives in ``gdn2_ref.c`` (one token at a time, fp64); this module 
 that file with gcc and marshals numpy arrays to it through ctypes. Which passage of the
 pages each step follows is stated in ``gdn2_ref.c``.
 
+``prologue_ref`` states the fused pre-processing (raw projections to q, k, log_alpha, b, w)
+in numpy, fp64; ``tests/test_oracle_prologue.py`` pins it.
+
 Parity status: every step is pinned by ``tests/test_oracle_pins.py`` (the delta-rule post's
 worked example, closed forms, invariants and brute force); the one reading the pages leave
 open -- which side of the erase term carries b -- is pinned to the adopted form only by a
@@ -114,3 +117,32 @@ def fwd_ref(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
     if rc != 0:
         raise ValueError(f"gdn2_fwd_ref rejected its arguments (status {rc})")
     return o, st
+
+
+def _f64(x):
+    if hasattr(x, "detach"):
+        return x.detach().double().cpu().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def prologue_ref(q_raw, k_raw, a_raw, b_raw, w_raw, eps: float = 1e-12):
+    """The fused pre-processing, fp64: from raw projections to the recurrence's inputs.
+
+      q = q_raw / max(|q_raw|_2, eps), k likewise, per token and head over the key axis.
+          The delta-rule post (ai-systems-engineering.com, section on the correction
+          strength beta) notes that re-reading the correction with the same key scales it by
+          k^T k, so the edit lands exactly only for unit-length keys.
+      log_alpha = -softplus(a_raw) = -log(1 + e^a): a decay alpha = 1 / (1 + e^a) in (0, 1).
+      b = sigmoid(b_raw), w = sigmoid(w_raw): gates in (0, 1), computed from the input (the
+          same section: the strength is produced from the input rather than fixed).
+    The pages name no activation functions; softplus and sigmoid are the reading adopted
+    here. Inputs: q_raw, k_raw [T, Hqk, dk]; a_raw, b_raw [T, Hv, dk]; w_raw [T, Hv, dv]
+    (torch tensors or arrays). Returns float64 arrays (q, k, log_alpha, b, w)."""
+    q, k, a, b, w = (_f64(x) for x in (q_raw, k_raw, a_raw, b_raw, w_raw))
+    qn = q / np.maximum(np.sqrt(np.sum(q * q, axis=-1, keepdims=True)), eps)
+    kn = k / np.maximum(np.sqrt(np.sum(k * k, axis=-1, keepdims=True)), eps)
+    log_alpha = -np.logaddexp(0.0, a)
+    with np.errstate(over="ignore"):
+        bs = 1.0 / (1.0 + np.exp(-b))
+        ws = 1.0 / (1.0 + np.exp(-w))
+    return qn, kn, log_alpha, bs, ws
