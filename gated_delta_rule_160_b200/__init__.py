@@ -60,6 +60,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdn2_decode_multi.restype = ctypes.c_int
     lib.gdn2_decode_multi.argtypes = ([ctypes.POINTER(Shape), ctypes.c_int] + [vp] * 8
                                       + [ctypes.c_int, vp, vp, vp])
+    lib.gdn2_decode_multi_prologue.restype = ctypes.c_int
+    lib.gdn2_decode_multi_prologue.argtypes = lib.gdn2_decode_multi.argtypes
+    lib.gdn2_chunk_fwd_prologue.restype = ctypes.c_int
+    lib.gdn2_chunk_fwd_prologue.argtypes = lib.gdn2_chunk_fwd.argtypes
     lib.gdn2_last_error_string.restype = ctypes.c_char_p
     lib.gdn2_last_error_string.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -103,13 +107,16 @@ def gdn2_chunk_fwd_workspace_size(shape: Shape, varlen: bool) -> int:
 
 def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None,
                    o=None, S_T=None, want_state: bool = True, workspace=None, stream=None,
-                   out_dtype=torch.float32):
+                   out_dtype=torch.float32, prologue: bool = False):
     """Prefill: run the recurrence over whole (packed) sequences on the GPU.
 
     q,k [T,Hqk,dk]; v,w [T,Hv,dv]; log_alpha (fp32), b [T,Hv,dk]; S0 fp32 [N,Hv,dk,dv] or
     None; cu_seqlens int32 [N+1] or None (then ``n_seq`` equal sequences, default 1).
     Returns (o [T,Hv,dv] in ``out_dtype`` (or o's dtype when given), S_T fp32 [N,Hv,dk,dv] or
     None). Tensors must be contiguous CUDA tensors; nothing is converted or copied here.
+    With ``prologue=True`` q, k, b, w are raw projections and ``log_alpha`` holds the decay
+    pre-activation a (same dtype as q): the kernel L2-normalises q and k, takes
+    log_alpha = -softplus(a) and sigmoid b, w (gdn2_chunk_fwd_prologue).
     """
     lib = load_library()
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
@@ -125,9 +132,10 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=Non
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.gdn2_chunk_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                              _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
-                              _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    fn = lib.gdn2_chunk_fwd_prologue if prologue else lib.gdn2_chunk_fwd
+    _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+              _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
+              _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
     return o, S_T
 
 
@@ -163,13 +171,14 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None, out_dtype
 
 
 def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_steps=None,
-                      want_steps: bool = False, stream=None, out_dtype=torch.float32):
+                      want_steps: bool = False, stream=None, out_dtype=torch.float32, prologue: bool = False):
     """Serving decode: n_tok new tokens for each of N sequences whose states sit in a pool.
 
     q,k [N,n_tok,Hqk,dk]; v,w [N,n_tok,Hv,dv]; log_alpha (fp32), b [N,n_tok,Hv,dk];
     S_pool fp32 [n_slots,Hv,dk,dv], updated in place; slots int32 [N] (slot of each
     sequence; negative = inactive, skipped) or None (slot n). Returns (o [N,n_tok,Hv,dv],
-    S_steps fp32 [N,n_tok,Hv,dk,dv] -- the state after each token -- or None)."""
+    S_steps fp32 [N,n_tok,Hv,dk,dv] -- the state after each token -- or None). ``prologue`` as
+    for gdn2_chunk_fwd (gdn2_decode_multi_prologue)."""
     lib = load_library()
     if o is not None:
         out_dtype = o.dtype
@@ -181,7 +190,8 @@ def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_st
         o = torch.empty((N, n_tok, h_v, dv), dtype=out_dtype, device=v.device)
     if S_steps is None and want_steps:
         S_steps = torch.empty((N, n_tok, h_v, dk, dv), dtype=torch.float32, device=v.device)
-    _check(lib.gdn2_decode_multi(ctypes.byref(shape), int(n_tok), _ptr(slots), _ptr(q), _ptr(k), _ptr(v),
-                                 _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
-                                 _ptr(o), _ptr(S_steps), _stream_handle(stream)))
+    fn = lib.gdn2_decode_multi_prologue if prologue else lib.gdn2_decode_multi
+    _check(fn(ctypes.byref(shape), int(n_tok), _ptr(slots), _ptr(q), _ptr(k), _ptr(v),
+              _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
+              _ptr(o), _ptr(S_steps), _stream_handle(stream)))
     return o, S_steps

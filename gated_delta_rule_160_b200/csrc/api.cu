@@ -113,16 +113,21 @@ size_t gdn2_chunk_fwd_workspace_size(const gdn2_shape* shape, int varlen) {
     return ((size_t)shape->n_seq * sizeof(int32_t) + 255) & ~(size_t)255;
 }
 
-gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k, const void* v,
-                           const float* log_alpha, const void* b, const void* w, const float* S0,
-                           const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
-                           size_t workspace_bytes, gdn2_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// gdn2_chunk_fwd and gdn2_chunk_fwd_prologue: with prologue, la is the dtype decay
+// pre-activation instead of fp32 log_alpha.
+gdn2_status chunk_fwd(bool prologue, const gdn2_shape* shape, const void* q, const void* k, const void* v,
+                      const void* la, const void* b, const void* w, const float* S0, const int32_t* cu_seqlens,
+                      void* o, float* S_T, void* workspace, size_t workspace_bytes, gdn2_stream_t stream) {
     gdn2_status st = check_shape(shape);
     if (st != GDN2_OK) return st;
     const bool any_tokens = shape->T_total > 0;
     const NamedPtr ps[] = {
         {"q", q, any_tokens}, {"k", k, any_tokens}, {"v", v, any_tokens},
-        {"log_alpha", log_alpha, any_tokens}, {"b", b, any_tokens}, {"w", w, any_tokens},
+        {prologue ? "a" : "log_alpha", la, any_tokens}, {"b", b, any_tokens}, {"w", w, any_tokens},
         {"o", o, any_tokens}, {"S0", S0, false}, {"S_T", S_T, false},
         {"cu_seqlens", cu_seqlens, false}, {"workspace", workspace, false},
     };
@@ -138,7 +143,12 @@ gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return fail(GDN2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
 
-    Params p = make_params(shape, q, k, v, log_alpha, b, w, S0, cu_seqlens, o, S_T);
+    Params p = make_params(shape, q, k, v, prologue ? nullptr : static_cast<const float*>(la), b, w, S0,
+                           cu_seqlens, o, S_T);
+    p.prologue = prologue;
+    p.a_raw = prologue ? la : nullptr;
+    if (prologue && any_tokens && !chunk_tc_supported(p, shape->dtype))
+        return fail(GDN2_ERR_UNSUPPORTED, "the fused pre-processing needs bf16 inputs with dk = dv = 128");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cu_seqlens) {
         int32_t* order = static_cast<int32_t*>(workspace);
@@ -150,6 +160,26 @@ gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k
                                                         : launch_recurrent(p, shape->dtype, shape->o_dtype, s);
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "chunk kernel launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn2_status gdn2_chunk_fwd(const gdn2_shape* shape, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const void* b, const void* w, const float* S0,
+                           const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
+                           size_t workspace_bytes, gdn2_stream_t stream) {
+    return chunk_fwd(false, shape, q, k, v, log_alpha, b, w, S0, cu_seqlens, o, S_T, workspace, workspace_bytes,
+                     stream);
+}
+
+gdn2_status gdn2_chunk_fwd_prologue(const gdn2_shape* shape, const void* q_raw, const void* k_raw, const void* v,
+                                    const void* a_raw, const void* b_raw, const void* w_raw, const float* S0,
+                                    const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
+                                    size_t workspace_bytes, gdn2_stream_t stream) {
+    return chunk_fwd(true, shape, q_raw, k_raw, v, a_raw, b_raw, w_raw, S0, cu_seqlens, o, S_T, workspace,
+                     workspace_bytes, stream);
 }
 
 gdn2_status gdn2_decode_step(const gdn2_shape* shape, const void* q, const void* k, const void* v,
@@ -174,9 +204,13 @@ gdn2_status gdn2_decode_step(const gdn2_shape* shape, const void* q, const void*
     return ok();
 }
 
-gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t* slots, const void* q,
-                              const void* k, const void* v, const float* log_alpha, const void* b, const void* w,
-                              float* S_pool, int n_slots, void* o, float* S_steps, gdn2_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+gdn2_status decode_multi(bool prologue, const gdn2_shape* shape, int n_tok, const int32_t* slots, const void* q,
+                         const void* k, const void* v, const void* la, const void* b, const void* w, float* S_pool,
+                         int n_slots, void* o, float* S_steps, gdn2_stream_t stream) {
     gdn2_status st = check_shape(shape);
     if (st != GDN2_OK) return st;
     if (n_tok < 1 || n_tok > GDN2_DECODE_MAX_TOKENS)
@@ -190,13 +224,16 @@ gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t*
     if ((long long)shape->n_seq * shape->h_v > 0x7fffffffLL || (long long)n_slots * shape->h_v > 0x7fffffffLL)
         return fail(GDN2_ERR_UNSUPPORTED, "n_seq * h_v or n_slots * h_v too large for one launch");
     const NamedPtr ps[] = {
-        {"q", q, true}, {"k", k, true}, {"v", v, true}, {"log_alpha", log_alpha, true}, {"b", b, true},
+        {"q", q, true}, {"k", k, true}, {"v", v, true}, {prologue ? "a" : "log_alpha", la, true}, {"b", b, true},
         {"w", w, true}, {"S_pool", S_pool, true}, {"o", o, true}, {"slots", slots, false},
         {"S_steps", S_steps, false},
     };
     st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
     if (st != GDN2_OK) return st;
-    Params p = make_params(shape, q, k, v, log_alpha, b, w, nullptr, nullptr, o, S_pool);
+    Params p = make_params(shape, q, k, v, prologue ? nullptr : static_cast<const float*>(la), b, w, nullptr,
+                           nullptr, o, S_pool);
+    p.prologue = prologue;
+    p.a_raw = prologue ? la : nullptr;
     p.n_tok = n_tok;
     p.slots = slots;
     p.n_slots = n_slots;
@@ -204,6 +241,24 @@ gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t*
     cudaError_t e = launch_decode(p, shape->dtype, shape->o_dtype, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "decode kernel launch: %s", cudaGetErrorString(e));
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t* slots, const void* q,
+                              const void* k, const void* v, const float* log_alpha, const void* b, const void* w,
+                              float* S_pool, int n_slots, void* o, float* S_steps, gdn2_stream_t stream) {
+    return decode_multi(false, shape, n_tok, slots, q, k, v, log_alpha, b, w, S_pool, n_slots, o, S_steps, stream);
+}
+
+gdn2_status gdn2_decode_multi_prologue(const gdn2_shape* shape, int n_tok, const int32_t* slots, const void* q_raw,
+                                       const void* k_raw, const void* v, const void* a_raw, const void* b_raw,
+                                       const void* w_raw, float* S_pool, int n_slots, void* o, float* S_steps,
+                                       gdn2_stream_t stream) {
+    return decode_multi(true, shape, n_tok, slots, q_raw, k_raw, v, a_raw, b_raw, w_raw, S_pool, n_slots, o, S_steps,
+                        stream);
 }
 
 }  // extern "C"

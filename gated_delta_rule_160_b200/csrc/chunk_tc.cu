@@ -107,6 +107,7 @@ constexpr uint32_t OFF_WA = OFF_REG + 3 * kSmall;      // fp32 A [64][WS]
 constexpr uint32_t OFF_WT = OFF_WA + 64 * WS * 4;     // fp32 T [64][WS]
 constexpr uint32_t OFF_WM = OFF_WT + 64 * WS * 4;     // fp32 scratch [32][33]
 constexpr uint32_t OFF_RAW_LA = OFF_REG;              // fp32, 32 KB  (group A)
+constexpr uint32_t OFF_RAW_A = OFF_REG + kTile;       // bf16 decay pre-activations (fused pre-processing)
 constexpr uint32_t OFF_RAW_V = OFF_REG + 2 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
 // float gref[2][128], glast[2][128], frame factors f[2][128], quarter-chunk log-decay
@@ -195,7 +196,11 @@ __device__ __forceinline__ void store8_bf16(uint8_t* smem, uint32_t off, const f
 template <typename TO>
 constexpr bool kTmaStoreO = sizeof(TO) == 4;  // the o tensor map is fp32
 
-template <typename TO>
+// kPro: fused pre-processing. The raw q, k are L2-normalised per token (norms over the 128
+// channels, reduced across the eight warps of a token through shared memory), log_alpha is
+// -softplus of the bf16 decay pre-activation (staged as a bf16 tile beside the cumulative
+// decay), b and w are sigmoids of their raw values.
+template <typename TO, bool kPro>
 __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__ Params p,
                                                           const __grid_constant__ RawMaps maps) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -248,11 +253,17 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const int c0 = 16 * (warp & 7) + 4 * (lane >> 3);
 
     // raw inputs of a chunk in two groups, each issued as soon as its space frees up
-    auto issue_raw_a = [&](int ts) {  // log_alpha, v, w
-        mbar_expect_tx(mbar(MB_RAWA), 4 * kTile);
+    auto issue_raw_a = [&](int ts) {  // log_alpha (or its bf16 pre-activation), v, w
+        mbar_expect_tx(mbar(MB_RAWA), kPro ? 3 * kTile : 4 * kTile);
+        if (kPro) {
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-            tma_load_3d(sbase + OFF_RAW_LA + x * 8192, &maps.la, 32 * x, h, ts, mbar(MB_RAWA));
+            for (int x = 0; x < 2; ++x)
+                tma_load_3d(sbase + OFF_RAW_A + x * 8192, &maps.la, 64 * x, h, ts, mbar(MB_RAWA));
+        } else {
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+                tma_load_3d(sbase + OFF_RAW_LA + x * 8192, &maps.la, 32 * x, h, ts, mbar(MB_RAWA));
+        }
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
             tma_load_3d(sbase + OFF_RAW_V + x * 8192, &maps.v, 64 * x, h, ts, mbar(MB_RAWA));
@@ -420,7 +431,28 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             // log_alpha rows: thread (channel c, quarter cp) sums tokens 16cp .. 16cp + 15 of
             // channel c. The totals of the earlier quarters are added where G is read.
             fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
-            {
+            if (kPro) {
+                // bf16 pre-activations a (upper half of the area), read completely before
+                // the cumulative decay overwrites the area
+                const int c = L;
+                float x[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const int i = 16 * cp + r;
+                    x[r] = i < nvalid ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                            smem + OFF_RAW_A + raw_off_bf16(i, c)))
+                                      : 0.f;
+                }
+                bar_sync_1<NS>();
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    const int i = 16 * cp + r;
+                    if (i < nvalid) acc = fmaf(-softplus_f(x[r]), kLog2e, acc);
+                    *reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c)) = acc;
+                }
+                qtot[128 * cp + c] = acc;
+            } else {
                 const int c = L;
                 float acc = 0.f;
 #pragma unroll
@@ -465,6 +497,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
                 bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
             }
+            if (kPro) {
+                // per-token partial sums of squares of q and k over this warp's 16 channels,
+                // into the T tile's space (idle during the prep): [token][channel group][q, k]
+                float* npart = reinterpret_cast<float*>(smem + OFF_T);
+#pragma unroll
+                for (int pss = 0; pss < 4; ++pss) {
+                    float qf[4], kf[4];
+                    unpack4_bf16(qq[pss], qf);
+                    unpack4_bf16(kq[pss], kf);
+                    float sq = qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3];
+                    float sk = kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3];
+#pragma unroll
+                    for (int off = 8; off < 32; off <<= 1) {  // the four channel quads of the token
+                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    }
+                    if (lane < 8)
+                        *reinterpret_cast<float2*>(npart + ((ti0 + 8 * pss) * 8 + (warp & 7)) * 2) = make_float2(sq, sk);
+                }
+            }
             // the tiles below overwrite the staged o tile (over Kb hi / lo) and Eb, which the
             // previous chunk's U -= R^T Eb MMAs read
             if (tid == 0) bulk_wait_read0();
@@ -472,6 +524,23 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             if (bar_or_1<NS>(fault)) {
                 fault = true;
                 break;
+            }
+            // 1 / |q|, 1 / |k| of this thread's tokens (all 128 channels)
+            float rq[4], rk[4];
+            if (kPro) {
+                const float4* npart = reinterpret_cast<const float4*>(smem + OFF_T);
+#pragma unroll
+                for (int pss = 0; pss < 4; ++pss) {
+                    float sq = 0.f, sk = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {  // eight channel groups, two per float4
+                        const float4 v = npart[(ti0 + 8 * pss) * 4 + j];
+                        sq += v.x + v.z;
+                        sk += v.y + v.w;
+                    }
+                    rq[pss] = __frcp_rn(fmaxf(sqrtf(sq), kL2NormEps));
+                    rk[pss] = __frcp_rn(fmaxf(sqrtf(sk), kL2NormEps));
+                }
             }
             // G - Gref: this thread's tokens lie in quarters 2th and 2th + 1, whose offsets
             // are the totals of the quarters before them
@@ -495,6 +564,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 unpack4_bf16(qq[pss], qf);
                 unpack4_bf16(kq[pss], kf);
                 unpack4_bf16(bq[pss], bf);
+                if (kPro) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        qf[e] *= rq[pss];
+                        kf[e] *= rk[pss];
+                        bf[e] = sigmoid_f(bf[e]);
+                    }
+                }
                 float kh[4], qv[4], kb[4], eb[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -538,6 +615,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             float vf[4], wf[4];
             unpack4_bf16(valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_V + ro) : z, vf);
             unpack4_bf16(valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_W + ro) : z, wf);
+            if (kPro) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) wf[e] = sigmoid_f(wf[e]);
+            }
             uint2 xh, xl;
             split2(wf[0] * vf[0], wf[1] * vf[1], xh.x, xl.x);
             split2(wf[2] * vf[2], wf[3] * vf[3], xh.y, xl.y);
@@ -890,12 +971,14 @@ bool encode_rows(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtensorMap* m, const voi
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename TO>
+template <typename TO, bool kPro>
 cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn) return cudaErrorNotSupported;
     RawMaps maps;
-    if (!encode_rows(fn, &maps.la, p.log_alpha, true, p.h_v, p.T_total, true) ||
+    const bool la_ok = kPro ? encode_rows(fn, &maps.la, p.a_raw, false, p.h_v, p.T_total, true)
+                            : encode_rows(fn, &maps.la, p.log_alpha, true, p.h_v, p.T_total, true);
+    if (!la_ok ||
         !encode_rows(fn, &maps.q, p.q, false, p.h_qk, p.T_total, true) ||
         !encode_rows(fn, &maps.k, p.k, false, p.h_qk, p.T_total, true) ||
         !encode_rows(fn, &maps.b, p.b, false, p.h_v, p.T_total, true) ||
@@ -908,10 +991,10 @@ cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
         maps.o = maps.la;  // unused: bf16 outputs take plain stores
     }
     // set on every launch: the attribute is per device and the call costs microseconds
-    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<TO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<TO, kPro>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    chunk_tc_kernel<TO><<<p.n_seq * p.h_v, NT, SMEM_BYTES, s>>>(p, maps);
+    chunk_tc_kernel<TO, kPro><<<p.n_seq * p.h_v, NT, SMEM_BYTES, s>>>(p, maps);
     return cudaGetLastError();
 }
 
@@ -922,7 +1005,8 @@ bool chunk_tc_supported(const Params& p, gdn2_dtype dt) {
 }
 
 cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s) {
-    return odt == GDN2_F32 ? launch_tc_t<float>(p, s) : launch_tc_t<__nv_bfloat16>(p, s);
+    if (p.prologue) return odt == GDN2_F32 ? launch_tc_t<float, true>(p, s) : launch_tc_t<__nv_bfloat16, true>(p, s);
+    return odt == GDN2_F32 ? launch_tc_t<float, false>(p, s) : launch_tc_t<__nv_bfloat16, false>(p, s);
 }
 
 cudaError_t read_tc_fault(unsigned int* out) {

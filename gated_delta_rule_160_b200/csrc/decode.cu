@@ -27,7 +27,9 @@ constexpr int kThreads = 256;
 // updated, which keeps fewer registers live (two CTAs per SM for dk = dv = 128). All the
 // tokens' inputs are staged in shared memory before the first one is applied, so HBM latency
 // is paid once per step, not once per token.
-template <int DK, int DV, typename T, typename TO, bool kMulti>
+// kPro: fused pre-processing (raw q, k L2-normalised per token; log_alpha = -softplus of
+// the decay pre-activation; sigmoid b, w), applied while the token inputs are staged.
+template <int DK, int DV, typename T, typename TO, bool kMulti, bool kPro>
 __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     constexpr int TPR = DV / 4;          // threads per state row
     constexpr int RG = kThreads / TPR;   // row groups
@@ -36,6 +38,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     __shared__ float sa[NTM][DK], sk[NTM][DK], sq[NTM][DK], se[NTM][DK], sx[NTM][DV];
     __shared__ float4 red[2][2][RG][TPR];  // [token parity][r | p]
     __shared__ float dots[NTM][2];
+    __shared__ float rnorm[NTM][2];  // 1 / |q|, 1 / |k| (fused pre-processing)
 
     const int item = blockIdx.x;  // n * h_v + h
     const int n = item / p.h_v;
@@ -60,33 +63,66 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
         const size_t row = (size_t)n * n_tok + t;
         const size_t tq = row * p.h_qk + g, tv = row * p.h_v + h;
         const float kv = to_f32(static_cast<const T*>(p.k)[tq * DK + c]);
+        const float bv = to_f32(static_cast<const T*>(p.b)[tv * DK + c]);
         sk[t][c] = kv;
         sq[t][c] = to_f32(static_cast<const T*>(p.q)[tq * DK + c]);
-        sa[t][c] = expf(p.log_alpha[tv * DK + c]);
-        se[t][c] = to_f32(static_cast<const T*>(p.b)[tv * DK + c]) * kv;
+        if (kPro) {  // alpha = exp(-softplus(a)) = 1 / (1 + e^a)
+            sa[t][c] = sigmoid_f(-to_f32(static_cast<const T*>(p.a_raw)[tv * DK + c]));
+            se[t][c] = sigmoid_f(bv) * kv;
+        } else {
+            sa[t][c] = expf(p.log_alpha[tv * DK + c]);
+            se[t][c] = bv * kv;
+        }
     }
     for (int idx = threadIdx.x; idx < n_tok * DV; idx += kThreads) {
         const int t = idx / DV, c = idx % DV;
         const size_t tv = ((size_t)n * n_tok + t) * p.h_v + h;
-        sx[t][c] = to_f32(static_cast<const T*>(p.w)[tv * DV + c]) * to_f32(static_cast<const T*>(p.v)[tv * DV + c]);
+        float wv = to_f32(static_cast<const T*>(p.w)[tv * DV + c]);
+        if (kPro) wv = sigmoid_f(wv);
+        sx[t][c] = wv * to_f32(static_cast<const T*>(p.v)[tv * DV + c]);
     }
     __syncthreads();
-    // q . (b (.) k) and q . k of every token: warp t takes token t
+    // q . (b (.) k) and q . k of every token (and |q|, |k| with the fused pre-processing):
+    // warp t takes token t
     for (int t = warp; t < n_tok; t += kThreads / 32) {
-        float d1 = 0.f, d2 = 0.f;
+        float d1 = 0.f, d2 = 0.f, nq = 0.f, nk = 0.f;
         for (int c = lane; c < DK; c += 32) {
             d1 += sq[t][c] * se[t][c];
             d2 += sq[t][c] * sk[t][c];
+            if (kPro) {
+                nq += sq[t][c] * sq[t][c];
+                nk += sk[t][c] * sk[t][c];
+            }
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
             d1 += __shfl_xor_sync(0xffffffffu, d1, off);
             d2 += __shfl_xor_sync(0xffffffffu, d2, off);
+            if (kPro) {
+                nq += __shfl_xor_sync(0xffffffffu, nq, off);
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+            }
         }
         if (lane == 0) {
-            dots[t][0] = d1;
-            dots[t][1] = d2;
+            float s2 = 1.f;
+            if (kPro) {
+                rnorm[t][0] = 1.f / fmaxf(sqrtf(nq), kL2NormEps);
+                rnorm[t][1] = 1.f / fmaxf(sqrtf(nk), kL2NormEps);
+                s2 = rnorm[t][0] * rnorm[t][1];
+            }
+            dots[t][0] = d1 * s2;
+            dots[t][1] = d2 * s2;
         }
+    }
+    if (kPro) {  // normalise the staged q, k (and b (.) k)
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < n_tok * DK; idx += kThreads) {
+            const int t = idx / DK, c = idx % DK;
+            sq[t][c] *= rnorm[t][0];
+            sk[t][c] *= rnorm[t][1];
+            se[t][c] *= rnorm[t][1];
+        }
+        __syncthreads();
     }
 
     // the state stays in registers from token to token
@@ -145,13 +181,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
     }
 }
 
+template <int DK, int DV, typename T, typename TO, bool kPro>
+cudaError_t launch_dec_p(const Params& p, cudaStream_t st) {
+    if (p.n_tok > 1 || p.S_steps)
+        decode_kernel<DK, DV, T, TO, true, kPro><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
+    else
+        decode_kernel<DK, DV, T, TO, false, kPro><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
 template <int DK, int DV, typename T, typename TO>
 cudaError_t launch_dec(const Params& p, cudaStream_t st) {
-    if (p.n_tok > 1 || p.S_steps)
-        decode_kernel<DK, DV, T, TO, true><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
-    else
-        decode_kernel<DK, DV, T, TO, false><<<p.n_seq * p.h_v, kThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    return p.prologue ? launch_dec_p<DK, DV, T, TO, true>(p, st) : launch_dec_p<DK, DV, T, TO, false>(p, st);
 }
 
 template <typename T, typename TO>

@@ -29,7 +29,24 @@ struct Params {
     const int32_t* slots;      // nullable: state slot of each sequence in S_T's pool
     int n_slots;               // states in the pool
     float* S_steps;            // nullable: state after each token [n_seq, n_tok, h_v, dk, dv]
+    // fused pre-processing: q, k, b, w are raw projections and log_alpha is replaced by the
+    // decay pre-activation a_raw (dtype, same layout): q, k <- L2-normalised, log_alpha <-
+    // -softplus(a_raw), b, w <- sigmoid
+    int prologue;
+    const void* a_raw;
 };
+
+// Pieces of the fused pre-processing, in fp32, on the special-function unit. Their errors
+// are absolute ~1e-7 (softplus: summed into log-decays) and relative ~1e-6 (sigmoid), far
+// below what the bf16 operands of the recurrence carry.
+__device__ __forceinline__ float sigmoid_f(float x) {
+    // 1 / (1 + e^-x); the exponent is capped where the quotient is already ~1e-35
+    return __fdividef(1.f, 1.f + __expf(fminf(-x, 80.f)));
+}
+__device__ __forceinline__ float softplus_f(float x) {  // log(1 + e^x), without overflow
+    return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
+}
+constexpr float kL2NormEps = 1e-12f;  // q and k are divided by max(|x|_2, eps)
 
 // Token range [t0, t1) of sequence n.
 __device__ __forceinline__ void seq_bounds(const Params& p, int n, int& t0, int& t1) {
@@ -56,7 +73,7 @@ cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cud
 cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s);
 cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s);
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt);
-cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);
+cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);  // honours p.prologue
 cudaError_t read_tc_fault(unsigned int* out);
 // Record a failure in the calling thread's error string and return st.
 gdn2_status report_error(gdn2_status st, const char* msg);

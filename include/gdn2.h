@@ -143,6 +143,39 @@ GDN2_API gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const
                               gdn2_stream_t stream);
 
 /*
+ * gdn2_decode_multi with the pre-processing of gdn2_chunk_fwd_prologue fused in (raw q, k,
+ * b, w; a_raw in dtype in place of log_alpha). Any dk, dv of the decode kernel.
+ */
+GDN2_API gdn2_status gdn2_decode_multi_prologue(const gdn2_shape* shape, int n_tok, const int32_t* slots,
+                                       const void* q_raw, const void* k_raw, const void* v,
+                                       const void* a_raw, const void* b_raw, const void* w_raw,
+                                       float* S_pool, int n_slots, void* o, float* S_steps,
+                                       gdn2_stream_t stream);
+
+/*
+ * Prefill with the pre-processing fused in: the inputs are raw projections, and the kernel
+ * applies, in fp32, per token and head,
+ *   q = q_raw / max(|q_raw|_2, 1e-12), k = k_raw / max(|k_raw|_2, 1e-12)   (over dk)
+ *   log_alpha = -softplus(a_raw) = -log(1 + e^a_raw)                        (per key channel)
+ *   b = sigmoid(b_raw), w = sigmoid(w_raw)
+ * before the recurrence above. Unit-length keys are what the delta-rule post
+ * (ai-systems-engineering.com, section on the correction strength beta) needs for the
+ * correction to land exactly, and gates computed from the input are what it describes; the
+ * activation functions themselves are not on the pages (softplus and sigmoid are the
+ * reading adopted). a_raw has dtype (not float32) and log_alpha's layout [T_total, h_v, dk];
+ * q_raw, k_raw, b_raw, w_raw replace q, k, b, w with the same layouts. Otherwise as
+ * gdn2_chunk_fwd (same workspace). Supported for bf16 inputs with dk = dv = 128 (else
+ * GDN2_ERR_UNSUPPORTED).
+ */
+GDN2_API gdn2_status gdn2_chunk_fwd_prologue(const gdn2_shape* shape,
+                                    const void* q_raw, const void* k_raw, const void* v,
+                                    const void* a_raw, const void* b_raw, const void* w_raw,
+                                    const float* S0, const int32_t* cu_seqlens,
+                                    void* o, float* S_T,
+                                    void* workspace, size_t workspace_bytes,
+                                    gdn2_stream_t stream);
+
+/*
  * Prefill for callers that cannot allocate device memory. The pages have no counterpart:
  * this is an interface choice. It computes exactly what gdn2_chunk_fwd computes (same
  * kernels, same arguments, no workspace), for callers that have no way to give the
