@@ -146,3 +146,60 @@ def prologue_ref(q_raw, k_raw, a_raw, b_raw, w_raw, eps: float = 1e-12):
         bs = 1.0 / (1.0 + np.exp(-b))
         ws = 1.0 / (1.0 + np.exp(-w))
     return qn, kn, log_alpha, bs, ws
+
+
+def _recurrence_torch(q, k, v, log_alpha, b, w, S0):
+    """The recurrence for one sequence in plain torch ops (fp64), token by token, as the
+    note on Gated DeltaNet-2 (section "Gated DeltaNet-2 design point") orders its steps:
+    decay on the key axis, key read of the decayed state, erase with b on the key axis,
+    write with w on the value axis; the delta-rule post has the query read the updated
+    state. Shapes: q, k [T, H, dk]; v, w [T, H, dv]; log_alpha, b [T, H, dk]; S0 [H, dk, dv]
+    (value heads H; q and k already expanded to them). Returns (o [T, H, dv], S_T)."""
+    import torch
+    S = S0
+    outs = []
+    for t in range(q.shape[0]):
+        S = torch.exp(log_alpha[t])[:, :, None] * S                       # S' = Diag(alpha) S
+        r = torch.einsum("hc,hcm->hm", k[t], S)                           # r = S'^T k
+        S = S - (b[t] * k[t])[:, :, None] * r[:, None, :] + k[t][:, :, None] * (w[t] * v[t])[:, None, :]
+        outs.append(torch.einsum("hc,hcm->hm", q[t], S))                  # o = S^T q
+    return torch.stack(outs), S
+
+
+def bwd_ref(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, n_seq=None):
+    """Gradients of the recurrence by reverse-mode differentiation of its plain fp64
+    statement (_recurrence_torch): the loss is sum(o * dO) + sum(S_T * dS_T).
+
+    Shapes as for fwd_ref (q, k [T, Hqk, dk]; v, w [T, Hv, dv]; log_alpha, b [T, Hv, dk];
+    S0, dS_T [N, Hv, dk, dv] or None; dO [T, Hv, dv]). Returns float64 arrays
+    (dq, dk [T, Hqk, dk]; dv, dw [T, Hv, dv]; dlog_alpha, db [T, Hv, dk]; dS0 [N, Hv, dk, dv]).
+    A query/key head's gradient sums over the value heads that read it. Small sizes only."""
+    import torch
+    f = lambda x: torch.as_tensor(_f64(x))
+    q, k, v, la, b, w, dO = (f(x).requires_grad_(True) if i < 6 else f(x)
+                             for i, x in enumerate((q, k, v, log_alpha, b, w, dO)))
+    T, h_qk, dk = q.shape
+    _, h_v, dv = v.shape
+    grp = h_v // h_qk
+    if cu_seqlens is not None:
+        cu = [int(c) for c in np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens)]
+    else:
+        n = 1 if n_seq is None else int(n_seq)
+        cu = [i * (T // n) for i in range(n + 1)]
+    N = len(cu) - 1
+    S0_t = (f(S0) if S0 is not None else torch.zeros(N, h_v, dk, dv, dtype=torch.float64)).requires_grad_(True)
+    loss = 0.0
+    for n in range(N):
+        s, e = cu[n], cu[n + 1]
+        qe = q[s:e].repeat_interleave(grp, dim=1)
+        ke = k[s:e].repeat_interleave(grp, dim=1)
+        if e > s:
+            o, S_T = _recurrence_torch(qe, ke, v[s:e], la[s:e], b[s:e], w[s:e], S0_t[n])
+            loss = loss + (o * dO[s:e]).sum()
+        else:
+            S_T = S0_t[n]
+        if dS_T is not None:
+            loss = loss + (S_T * f(dS_T)[n]).sum()
+    grads = torch.autograd.grad(loss, (q, k, v, la, b, w, S0_t), allow_unused=True)
+    return tuple(np.zeros(x.shape) if g_ is None else g_.numpy()
+                 for g_, x in zip(grads, (q, k, v, la, b, w, S0_t)))
