@@ -16,6 +16,7 @@ workload on this host's cores.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -34,6 +35,7 @@ PREFILL = "prefill_b8_h16_t4096"
 DECODE = "decode_256seq_h32"
 SERVING_TOKENS = 4  # tokens per sequence in one serving-decode step (a verify step)
 PROLOGUE_TIMED_STEPS = 10
+BACKWARD_TIMED_STEPS = 3
 DECODE_TIMED_STEPS = 64
 
 
@@ -149,6 +151,17 @@ def prologue_bytes(wl, lengths) -> int:
     per_token = wl.h_qk * 2 * wl.dk * es + wl.h_v * (2 * wl.dv * es + 2 * wl.dk * es + 4 * wl.dv)
     state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
     return T * per_token + state * (2 if wl.S0_std else 1)
+
+
+def backward_bytes(wl, lengths) -> int:
+    """Algorithmic bytes of one backward: the forward's inputs and dO read once, every
+    gradient (fp32) written once, S0 read and dS0 written."""
+    es = torch.finfo(wl.dtype).bits // 8
+    T = int(sum(lengths))
+    reads = wl.h_qk * 2 * wl.dk * es + wl.h_v * (2 * wl.dv * es + wl.dk * es + 4 * wl.dk + 4 * wl.dv)
+    writes = wl.h_qk * 2 * wl.dk * 4 + wl.h_v * (2 * wl.dv * 4 + 2 * wl.dk * 4)
+    state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
+    return T * (reads + writes) + state * 2
 
 
 def serving_bytes(wl, n_tok: int) -> int:
@@ -334,6 +347,33 @@ def main():
                              "algorithmic_bytes_per_launch": pbytes}}
     del raw
 
+    # ---------------- backward (gradients of sum(o * dO)), same workload
+    dO_b = torch.randn(o.shape, generator=torch.Generator(device=dev).manual_seed(wl.seed + 29), device=dev)
+    sh_b = G.make_shape(d["q"], d["v"], d["n_seq"], torch.float32)
+    ws_b = torch.empty(int(G.load_library().gdn2_chunk_bwd_workspace_size(ctypes.byref(sh_b))),
+                       dtype=torch.uint8, device=dev)
+    bstep = lambda: G.gdn2_chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], dO_b, S0=d["S0"],
+                                     n_seq=d["n_seq"], workspace=ws_b, stream=stream)
+    bstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(BACKWARD_TIMED_STEPS):
+        bstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bms = max_over_ranks(e0.elapsed_time(e1) / BACKWARD_TIMED_STEPS, world)
+    bbytes = backward_bytes(wl, d["lengths"])
+    bach = bbytes / (bms / 1000.0) / 1e9
+    backward = {"metric": "GDN-2 backward tokens/s", "value": world * T_all / (bms / 1000.0), "unit": "tokens/s",
+                "ms_per_step": bms, "steps": BACKWARD_TIMED_STEPS,
+                "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (first, sequential form)"},
+                "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
+                             "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                             "algorithmic_bytes_per_launch": bbytes}}
+    del dO_b, ws_b
+
     # ---------------- decode (the second metric)
     dwl = W.WORKLOADS[DECODE]
     S = W.decode_state(dwl, dev)
@@ -453,6 +493,7 @@ def main():
             "decode": decode,
             "serving_decode": serving,
             "prefill_prologue": prologue,
+            "backward": backward,
             "e2e": e2e,
             "cpu_baseline": base,
             "clocks": clocks.summary(),

@@ -64,6 +64,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdn2_decode_multi_prologue.argtypes = lib.gdn2_decode_multi.argtypes
     lib.gdn2_chunk_fwd_prologue.restype = ctypes.c_int
     lib.gdn2_chunk_fwd_prologue.argtypes = lib.gdn2_chunk_fwd.argtypes
+    lib.gdn2_chunk_bwd_workspace_size.restype = sz
+    lib.gdn2_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
+    lib.gdn2_chunk_bwd.restype = ctypes.c_int
+    lib.gdn2_chunk_bwd.argtypes = [ctypes.POINTER(Shape)] + [vp] * 17 + [vp, sz, vp]
     lib.gdn2_last_error_string.restype = ctypes.c_char_p
     lib.gdn2_last_error_string.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -195,3 +199,26 @@ def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_st
               _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
               _ptr(o), _ptr(S_steps), _stream_handle(stream)))
     return o, S_steps
+
+
+def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=None, n_seq=None,
+                   want_dS0: bool = True, workspace=None, stream=None):
+    """Gradients of sum(o * dO) + sum(S_T * dS_T) with respect to the forward's inputs.
+    Shapes as for gdn2_chunk_fwd; dO fp32 [T,Hv,dv]. Returns fp32 tensors
+    (dq, dk, dv, dlog_alpha, db, dw, dS0 or None)."""
+    lib = load_library()
+    n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
+    shape = make_shape(q, v, n, torch.float32)
+    dev = v.device
+    f = lambda t: torch.empty(t.shape, dtype=torch.float32, device=dev)
+    dq, dk, dv, dla, db, dw = f(q), f(k), f(v), f(log_alpha), f(b), f(w)
+    dS0 = torch.empty((n, v.shape[1], q.shape[2], v.shape[2]), dtype=torch.float32, device=dev) if want_dS0 else None
+    need = int(lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(shape)))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.gdn2_chunk_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                              _ptr(S0), _ptr(cu_seqlens), _ptr(dO), _ptr(dS_T), _ptr(dq), _ptr(dk), _ptr(dv),
+                              _ptr(dla), _ptr(db), _ptr(dw), _ptr(dS0), _ptr(workspace),
+                              ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    return dq, dk, dv, dla, db, dw, dS0

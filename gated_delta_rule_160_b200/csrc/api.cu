@@ -261,4 +261,42 @@ gdn2_status gdn2_decode_multi_prologue(const gdn2_shape* shape, int n_tok, const
                         stream);
 }
 
+size_t gdn2_chunk_bwd_workspace_size(const gdn2_shape* shape) {
+    if (!shape || shape->n_seq < 1 || shape->T_total < 0 || shape->h_v < 1 || shape->dk < 1 || shape->dv < 1) return 0;
+    return (bwd_workspace_bytes(shape) + 255) & ~(size_t)255;
+}
+
+gdn2_status gdn2_chunk_bwd(const gdn2_shape* shape, const void* q, const void* k, const void* v,
+                           const float* log_alpha, const void* b, const void* w, const float* S0,
+                           const int32_t* cu_seqlens, const float* dO, const float* dS_T, float* dq, float* dk,
+                           float* dv, float* dlog_alpha, float* db, float* dw, float* dS0, void* workspace,
+                           size_t workspace_bytes, gdn2_stream_t stream) {
+    gdn2_status st = check_shape(shape);
+    if (st != GDN2_OK) return st;
+    const bool any = shape->T_total > 0;
+    const NamedPtr ps[] = {
+        {"q", q, any}, {"k", k, any}, {"v", v, any}, {"log_alpha", log_alpha, any}, {"b", b, any},
+        {"w", w, any}, {"dO", dO, any}, {"dq", dq, any}, {"dk", dk, any}, {"dv", dv, any},
+        {"dlog_alpha", dlog_alpha, any}, {"db", db, any}, {"dw", dw, any}, {"S0", S0, false},
+        {"cu_seqlens", cu_seqlens, false}, {"dS_T", dS_T, false}, {"dS0", dS0, false},
+        {"workspace", workspace, false},
+    };
+    st = check_ptrs(ps, (int)(sizeof ps / sizeof ps[0]));
+    if (st != GDN2_OK) return st;
+    if (!cu_seqlens && shape->T_total % shape->n_seq != 0)
+        return fail(GDN2_ERR_INVALID_ARG, "T_total = %d is not a multiple of n_seq = %d (and no cu_seqlens)",
+                    shape->T_total, shape->n_seq);
+    const size_t need = gdn2_chunk_bwd_workspace_size(shape);
+    if (!workspace || workspace_bytes < need)
+        return fail(GDN2_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(GDN2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+    Params p = make_params(shape, q, k, v, log_alpha, b, w, S0, cu_seqlens, nullptr, nullptr);
+    cudaError_t e = launch_bwd(p, shape->dtype, dO, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0, workspace,
+                               reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "backward kernel launch: %s", cudaGetErrorString(e));
+    return ok();
+}
+
 }  // extern "C"

@@ -75,6 +75,10 @@ cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s)
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt);
 cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);  // honours p.prologue
 cudaError_t read_tc_fault(unsigned int* out);
+// Backward (gradients of the recurrence).
+size_t bwd_workspace_bytes(const gdn2_shape* sh);
+cudaError_t launch_bwd(const Params& p, gdn2_dtype dt, const float* dO, const float* dS_T, float* dq, float* dk,
+                       float* dv, float* dla, float* db, float* dw, float* dS0, void* workspace, cudaStream_t s);
 // Record a failure in the calling thread's error string and return st.
 gdn2_status report_error(gdn2_status st, const char* msg);
 

@@ -176,6 +176,34 @@ GDN2_API gdn2_status gdn2_chunk_fwd_prologue(const gdn2_shape* shape,
                                     gdn2_stream_t stream);
 
 /*
+ * Gradients of the recurrence for the loss L = sum(o * dO) + sum(S_T * dS_T): given the
+ * forward's inputs (as for gdn2_chunk_fwd) and dO [T_total, h_v, dv] float32 (dS_T nullable,
+ * [n_seq, h_v, dk, dv] float32), writes, all float32 and in the inputs' layouts,
+ *   dq, dk [T_total, h_qk, dk]  (a query/key head sums over the value heads that read it)
+ *   dv, dw [T_total, h_v, dv];  dlog_alpha, db [T_total, h_v, dk]
+ *   dS0 (nullable) [n_seq, h_v, dk, dv].
+ * The pages describe the forward recurrence only (they state the model was trained, which
+ * needs these); the derivation is the chain rule through the per-token update. This first
+ * form runs one CTA per (sequence, value head), sequentially: a forward pass storing the
+ * state at every 64th token, then, chunk by chunk from the end, the chunk's states are
+ * recomputed into a scratch area and its tokens walked backwards.
+ * workspace: device memory of gdn2_chunk_bwd_workspace_size(shape) bytes, 256-byte
+ * aligned (required). With h_v > h_qk, dq and dk are zeroed on the stream and accumulated
+ * with atomics (the order of those additions varies from run to run).
+ * Any dtype and dk, dv in {64, 128}.
+ */
+GDN2_API size_t gdn2_chunk_bwd_workspace_size(const gdn2_shape* shape);
+GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_shape* shape,
+                           const void* q, const void* k, const void* v,
+                           const float* log_alpha, const void* b, const void* w,
+                           const float* S0, const int32_t* cu_seqlens,
+                           const float* dO, const float* dS_T,
+                           float* dq, float* dk, float* dv,
+                           float* dlog_alpha, float* db, float* dw, float* dS0,
+                           void* workspace, size_t workspace_bytes,
+                           gdn2_stream_t stream);
+
+/*
  * Prefill for callers that cannot allocate device memory. The pages have no counterpart:
  * this is an interface choice. It computes exactly what gdn2_chunk_fwd computes (same
  * kernels, same arguments, no workspace), for callers that have no way to give the
