@@ -94,13 +94,32 @@ __device__ void forward_token(Smem<DK, DV>& sm) {
     __syncthreads();
 }
 
+// State copies between global memory ([DK][DV], contiguous) and the padded shared array:
+// 16-byte global accesses, every load of a thread issued before its first store.
 template <int DK, int DV>
 __device__ void store_state(const Smem<DK, DV>& sm, float* dst) {
-    for (int idx = threadIdx.x; idx < DK * DV; idx += kBT) dst[idx] = sm.S[idx / DV][idx % DV];
+    constexpr int N4 = DK * DV / 4 / kBT;
+#pragma unroll
+    for (int j = 0; j < N4; ++j) {
+        const int i4 = threadIdx.x + j * kBT, c = (4 * i4) / DV, m = (4 * i4) % DV;
+        reinterpret_cast<float4*>(dst)[i4] = make_float4(sm.S[c][m], sm.S[c][m + 1], sm.S[c][m + 2], sm.S[c][m + 3]);
+    }
 }
 template <int DK, int DV>
 __device__ void load_state(Smem<DK, DV>& sm, const float* src) {
-    for (int idx = threadIdx.x; idx < DK * DV; idx += kBT) sm.S[idx / DV][idx % DV] = src ? src[idx] : 0.f;
+    constexpr int N4 = DK * DV / 4 / kBT;
+    float4 r[N4];
+#pragma unroll
+    for (int j = 0; j < N4; ++j)
+        r[j] = src ? reinterpret_cast<const float4*>(src)[threadIdx.x + j * kBT] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < N4; ++j) {
+        const int i4 = threadIdx.x + j * kBT, c = (4 * i4) / DV, m = (4 * i4) % DV;
+        sm.S[c][m] = r[j].x;
+        sm.S[c][m + 1] = r[j].y;
+        sm.S[c][m + 2] = r[j].z;
+        sm.S[c][m + 3] = r[j].w;
+    }
 }
 
 template <int DK, int DV, typename T>
