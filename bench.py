@@ -368,7 +368,7 @@ def main():
     bach = bbytes / (bms / 1000.0) / 1e9
     backward = {"metric": "GDN-2 backward tokens/s", "value": world * T_all / (bms / 1000.0), "unit": "tokens/s",
                 "ms_per_step": bms, "steps": BACKWARD_TIMED_STEPS,
-                "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (first, sequential form)"},
+                "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (per-token adjoint, fp32, column slices per warp)"},
                 "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
                              "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
                              "algorithmic_bytes_per_launch": bbytes}}

@@ -1,4 +1,4 @@
-// backward.cu -- gradients of the recurrence (gdn2_chunk_bwd): a first, sequential form.
+// backward.cu -- gradients of the recurrence (gdn2_chunk_bwd).
 //
 // For each token, with e = b (.) k, x = w (.) v, S' = Diag(alpha) S_prev, r = S'^T k,
 // S = S' - e r^T + k x^T, o = S^T q, and the adjoint dS of S (from later tokens and dS_T):
@@ -7,284 +7,434 @@
 //   de   = -dS r,   dk = dS x + Diag(alpha) S_prev dr + de (.) b,   db = de (.) k
 //   dS'  = dS + k dr^T
 //   dalpha = rowsum(dS' (.) S_prev),  dlog_alpha = dalpha (.) alpha
-//   dq   = Diag(alpha) S_prev dO - e (r . dO) + k (x . dO)     (= S dO)
+//   dq   = S dO = Diag(alpha) S_prev dO - e (r . dO) + k (x . dO)
 //   dw   = dx (.) v,  dv = dx (.) w,  and the adjoint of S_prev is Diag(alpha) dS'.
-// One CTA per (sequence, value head). It runs the recurrence forward once, storing the
-// state at the start of every 64-token chunk; then, chunk by chunk from the last, it
-// recomputes the chunk's states from that checkpoint into a per-CTA scratch area and walks
-// the chunk's tokens backwards. S_prev and dS live in shared memory with rows padded to
-// DV + 1 floats, so that row sums (thread = row) and column sums (thread = column) are both
-// free of bank conflicts. A query/key head's dq, dk sum over the value heads that read it:
-// with groups of several value heads they are accumulated with atomics into outputs the
-// host zeroed first.
+//
+// Every value column of the state evolves on its own: the forward update and the adjoint of
+// column m read only column m and the token's key-side vectors. So one CTA per (sequence,
+// value head) gives each warp 16 value columns and keeps that dk x 16 slice of S_prev and of
+// dS in registers (lane l holds key rows l, l + 32, ...). Column sums (r, dx, dr) are a warp
+// reduction; the per-row gradients (dq, dk, db, dlog_alpha) are sums over all columns, so each
+// warp writes its partial row sums to shared memory and, after one barrier per token, the CTA
+// adds the warps' partials and writes the outputs.
+//
+// Forward, then backward, over sub-chunks of kL tokens: a first pass stores the state at the
+// start of every sub-chunk (checkpoints); then, from the last sub-chunk, the sub-chunk's states
+// are recomputed from its checkpoint into a per-CTA scratch area (small enough to stay in L2)
+// and its tokens are walked backwards. Each thread stores and reloads only its own slice of a
+// state, in its own register order, so these copies need no synchronisation; the next token's
+// S_prev is prefetched with cp.async into a per-thread double buffer while the current one is
+// processed. Token inputs are staged in shared memory a sub-chunk at a time, double-buffered.
+// A query/key head's dq, dk sum over the value heads that read it: with groups of several
+// value heads they are accumulated with atomics into outputs the host zeroed first.
 #include "internal.cuh"
 
 namespace gdn2 {
 namespace {
 
-constexpr int kBT = 256;     // threads per CTA
-constexpr int kCk = 64;      // tokens per checkpoint interval
+constexpr int kL = 8;        // tokens per sub-chunk (checkpoint interval)
+constexpr int kMC = 16;      // value columns per warp
 
 struct BwdParams {
     Params f;                // the forward's arguments
     const float* dO;         // [T, h_v, dv]
     const float* dS_T;       // nullable [N, h_v, dk, dv]
     float *dq, *dk, *dv, *dla, *db, *dw, *dS0;  // dS0 nullable
-    float* ckpt;             // [sum of chunks, h_v, dk, dv]
-    float* scratch;          // [N * h_v, kCk, dk, dv]
+    float4* ckpt;            // [slots, h_v, dk * dv / 4]; slot = n + t0 / kL + sub-chunk
+    float4* scratch;         // [N * h_v, kL - 1, dk * dv / 4]
     int atomic_qk;           // dq, dk accumulate (groups of value heads)
 };
 
-template <int DK, int DV>
-struct Smem {
-    float S[DK][DV + 1];     // S_prev (or the running state in the forward passes)
-    float dS[DK][DV + 1];    // adjoint of the state after the current token
-    float k[DK], q[DK], al[DK], e[DK], b[DK];
-    float x[DV], v[DV], w[DV], dO[DV], r[DV], dx[DV], dr[DV];
-    float cpart[kBT / DV][3][DV];  // column-sum partials (r, dx, dr)
-    float rpart[kBT / DK][5][DK];  // row-sum partials (de, dk, dalpha, S_prev dO, unused)
-    float dots[2];                 // r . dO, x . dO
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// 16 consecutive values (16-byte aligned) as fp32; a warp reading one address broadcasts.
+__device__ __forceinline__ void ld16(const float* p, float (&o)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float4 u = reinterpret_cast<const float4*>(p)[i];
+        o[4 * i] = u.x; o[4 * i + 1] = u.y; o[4 * i + 2] = u.z; o[4 * i + 3] = u.w;
+    }
+}
+__device__ __forceinline__ void ld16(const __nv_bfloat16* p, float (&o)[16]) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const uint4 u = reinterpret_cast<const uint4*>(p)[i];
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[j]));
+            o[8 * i + 2 * j] = f.x;
+            o[8 * i + 2 * j + 1] = f.y;
+        }
+    }
+}
+
+// Sums of a[v][0..15] over the warp's 32 lanes, NV vectors at once: each step hands half of
+// the remaining columns to the partner lane, so 8 + 4 + 2 + 1 + 1 shuffles per vector leave
+// in a[v][0] the full sum of column (lane >> 1).
+template <int NV>
+__device__ __forceinline__ void col_reduce(float (&a)[NV][16], int lane) {
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+        const int half = 8 >> st, xm = 16 >> st;
+        const bool up = lane & xm;
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float send = up ? a[v][i] : a[v][i + half];
+                const float keep = up ? a[v][i + half] : a[v][i];
+                a[v][i] = keep + __shfl_xor_sync(0xffffffffu, send, xm);
+            }
+    }
+#pragma unroll
+    for (int v = 0; v < NV; ++v) a[v][0] += __shfl_xor_sync(0xffffffffu, a[v][0], 1);
+}
+
+template <int DK, int DV, typename T>
+struct Cfg {
+    static constexpr int NW = DV / kMC, NT = 32 * NW, RJ = DK / 32;
+    static constexpr int ES = sizeof(T);
+    // one token's inputs in shared memory: k, q, b, v, w (dtype), log_alpha, dO (fp32)
+    static constexpr int OFF_K = 0, OFF_Q = DK * ES, OFF_B = 2 * DK * ES, OFF_V = 3 * DK * ES;
+    static constexpr int OFF_W = OFF_V + DV * ES, OFF_LA = OFF_W + DV * ES, OFF_DO = OFF_LA + 4 * DK;
+    static constexpr int REC = OFF_DO + 4 * DV;
+    static constexpr int CK = DK * ES / 16, CV = DV * ES / 16, CLA = DK / 4, CDO = DV / 4;
+    static constexpr int CPT = 3 * CK + 2 * CV + CLA + CDO;  // 16-byte pieces per token
+    static constexpr int S4 = DK * DV / 4;                   // float4 per state
+    // shared memory (bytes)
+    static constexpr int SM_TOK = 0;                              // [2][kL][REC]
+    static constexpr int SM_SP = SM_TOK + 2 * kL * REC;           // [2][S4] float4: S_prev
+    static constexpr int SM_PART = SM_SP + 2 * S4 * 16;           // [2][NW][4][DK] f32: row partials
+    static constexpr int SM_COL = SM_PART + 2 * NW * 4 * DK * 4;  // [NW][2][16] f32: r, dr
+    static constexpr int SMEM = SM_COL + NW * 2 * kMC * 4;
 };
 
-template <typename T>
-__device__ __forceinline__ float ld(const void* base, size_t i) {
-    return to_f32(static_cast<const T*>(base)[i]);
+// Queue (cp.async) the inputs of tokens [ts, ts + len) into a token buffer.
+template <int DK, int DV, typename T>
+__device__ void issue_tokens(const BwdParams& bp, uint8_t* dst, int ts, int len, int g, int h, bool with_dO) {
+    using C = Cfg<DK, DV, T>;
+    const Params& p = bp.f;
+    const int total = len * C::CPT;
+    for (int u = threadIdx.x; u < total; u += C::NT) {
+        const int i = u / C::CPT, r = u - i * C::CPT;
+        const size_t tok = (size_t)ts + i, rq = tok * p.h_qk + g, rv = tok * p.h_v + h;
+        const char* src;
+        if (r < 3 * C::CK) {
+            const int seg = r / C::CK, off = r - seg * C::CK;
+            const void* base = seg == 0 ? p.k : (seg == 1 ? p.q : p.b);
+            src = static_cast<const char*>(base) + (seg < 2 ? rq : rv) * (DK * C::ES) + off * 16;
+        } else if (r < 3 * C::CK + 2 * C::CV) {
+            const int r2 = r - 3 * C::CK, seg = r2 / C::CV, off = r2 - seg * C::CV;
+            src = static_cast<const char*>(seg == 0 ? p.v : p.w) + rv * (DV * C::ES) + off * 16;
+        } else if (r < 3 * C::CK + 2 * C::CV + C::CLA) {
+            src = reinterpret_cast<const char*>(p.log_alpha + rv * DK) + (r - 3 * C::CK - 2 * C::CV) * 16;
+        } else {
+            if (!with_dO) continue;
+            src = reinterpret_cast<const char*>(bp.dO + rv * DV) + (r - 3 * C::CK - 2 * C::CV - C::CLA) * 16;
+        }
+        cp_async16(dst + i * C::REC + r * 16, src);
+    }
+}
+
+// Key-side values of a token for this lane's rows.
+template <int RJ>
+struct RowVals {
+    float k[RJ], q[RJ], al[RJ], b[RJ], e[RJ];
+};
+template <int DK, int DV, typename T>
+__device__ __forceinline__ RowVals<DK / 32> row_vals(const uint8_t* rec, int lane) {
+    using C = Cfg<DK, DV, T>;
+    RowVals<DK / 32> rv;
+    const T* kt = reinterpret_cast<const T*>(rec + C::OFF_K);
+    const T* qt = reinterpret_cast<const T*>(rec + C::OFF_Q);
+    const T* bt = reinterpret_cast<const T*>(rec + C::OFF_B);
+    const float* lat = reinterpret_cast<const float*>(rec + C::OFF_LA);
+#pragma unroll
+    for (int j = 0; j < C::RJ; ++j) {
+        const int c = lane + 32 * j;
+        rv.k[j] = to_f32(kt[c]);
+        rv.q[j] = to_f32(qt[c]);
+        rv.b[j] = to_f32(bt[c]);
+        rv.al[j] = expf(lat[c]);
+        rv.e[j] = rv.b[j] * rv.k[j];
+    }
+    return rv;
+}
+
+// One forward token on this thread's slice S (key rows lane + 32 j, the warp's 16 columns).
+template <int DK, int DV, typename T>
+__device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t* rec, float* col, int lane,
+                                         int warp) {
+    using C = Cfg<DK, DV, T>;
+    const auto rv = row_vals<DK, DV, T>(rec, lane);
+    float a[1][16];
+#pragma unroll
+    for (int mm = 0; mm < 16; ++mm) {
+        float s = 0.f;
+#pragma unroll
+        for (int j = 0; j < C::RJ; ++j) s = fmaf(rv.al[j] * rv.k[j], S[j][mm], s);
+        a[0][mm] = s;
+    }
+    col_reduce<1>(a, lane);
+    __syncwarp();
+    if (!(lane & 1)) col[lane >> 1] = a[0][0];
+    __syncwarp();
+    float r[16], v[16], w[16];
+    ld16(col, r);
+    ld16(reinterpret_cast<const T*>(rec + C::OFF_V) + kMC * warp, v);
+    ld16(reinterpret_cast<const T*>(rec + C::OFF_W) + kMC * warp, w);
+#pragma unroll
+    for (int j = 0; j < C::RJ; ++j)
+#pragma unroll
+        for (int mm = 0; mm < 16; ++mm)
+            S[j][mm] = fmaf(rv.k[j], w[mm] * v[mm], fmaf(-rv.e[j], r[mm], rv.al[j] * S[j][mm]));
+}
+
+// A thread's slice of a state in its own order: float4 index of (row group j, column quad qq).
+template <int DK>
+__device__ __forceinline__ int sidx(int warp, int lane, int j, int qq) {
+    return warp * (DK / 32) * 128 + (j * 4 + qq) * 32 + lane;
+}
+template <int DK>
+__device__ __forceinline__ void put_slice(float4* dst, const float (&S)[DK / 32][kMC], int warp, int lane) {
+#pragma unroll
+    for (int j = 0; j < DK / 32; ++j)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+            dst[sidx<DK>(warp, lane, j, qq)] =
+                make_float4(S[j][4 * qq], S[j][4 * qq + 1], S[j][4 * qq + 2], S[j][4 * qq + 3]);
+}
+template <int DK>
+__device__ __forceinline__ void get_slice(float (&S)[DK / 32][kMC], const float4* src, int warp, int lane) {
+#pragma unroll
+    for (int j = 0; j < DK / 32; ++j)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const float4 u = src[sidx<DK>(warp, lane, j, qq)];
+            S[j][4 * qq] = u.x; S[j][4 * qq + 1] = u.y; S[j][4 * qq + 2] = u.z; S[j][4 * qq + 3] = u.w;
+        }
+}
+template <int DK>
+__device__ __forceinline__ void copy_slice_async(float4* dst, const float4* src, int warp, int lane) {
+#pragma unroll
+    for (int j = 0; j < DK / 32; ++j)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const int i = sidx<DK>(warp, lane, j, qq);
+            cp_async16(dst + i, src + i);
+        }
+}
+// The same slice in a [dk][dv] row-major state (S0, dS_T, dS0).
+template <int DV>
+__device__ __forceinline__ int gidx(int warp, int lane, int j, int qq) {
+    return ((lane + 32 * j) * DV + kMC * warp + 4 * qq) / 4;
+}
+template <int DK, int DV>
+__device__ __forceinline__ void load_rowmajor(float (&S)[DK / 32][kMC], const float* src, int warp, int lane) {
+#pragma unroll
+    for (int j = 0; j < DK / 32; ++j)
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const float4 u = src ? reinterpret_cast<const float4*>(src)[gidx<DV>(warp, lane, j, qq)]
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[j][4 * qq] = u.x; S[j][4 * qq + 1] = u.y; S[j][4 * qq + 2] = u.z; S[j][4 * qq + 3] = u.w;
+        }
 }
 
 template <int DK, int DV, typename T>
-__device__ void load_token(const Params& p, Smem<DK, DV>& sm, size_t tok, int g, int h, const float* dO) {
-    const size_t tq = tok * p.h_qk + g, tv = tok * p.h_v + h;
-    for (int c = threadIdx.x; c < DK; c += kBT) {
-        const float kv = ld<T>(p.k, tq * DK + c), bv = ld<T>(p.b, tv * DK + c);
-        sm.k[c] = kv;
-        sm.q[c] = ld<T>(p.q, tq * DK + c);
-        sm.al[c] = expf(p.log_alpha[tv * DK + c]);
-        sm.b[c] = bv;
-        sm.e[c] = bv * kv;
-    }
-    for (int m = threadIdx.x; m < DV; m += kBT) {
-        const float vv = ld<T>(p.v, tv * DV + m), wv = ld<T>(p.w, tv * DV + m);
-        sm.v[m] = vv;
-        sm.w[m] = wv;
-        sm.x[m] = wv * vv;
-        if (dO) sm.dO[m] = dO[tv * DV + m];
-    }
-}
+__global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const __grid_constant__ BwdParams bp) {
+    using C = Cfg<DK, DV, T>;
+    constexpr int RJ = C::RJ;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t* tok = smem + C::SM_TOK;
+    float4* spb = reinterpret_cast<float4*>(smem + C::SM_SP);
+    float* part = reinterpret_cast<float*>(smem + C::SM_PART);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* col = reinterpret_cast<float*>(smem + C::SM_COL) + warp * 2 * kMC;  // r, dr of the warp's columns
 
-// One forward token on sm.S (state in, state out); token vectors already loaded.
-template <int DK, int DV>
-__device__ void forward_token(Smem<DK, DV>& sm) {
-    constexpr int CP = kBT / DV;  // column parts
-    const int m = threadIdx.x % DV, part = threadIdx.x / DV;
-    float acc = 0.f;
-    for (int c = part; c < DK; c += CP) acc = fmaf(sm.al[c] * sm.k[c], sm.S[c][m], acc);
-    sm.cpart[part][0][m] = acc;
-    __syncthreads();
-    if (threadIdx.x < DV) {
-        float r = 0.f;
-#pragma unroll
-        for (int j = 0; j < CP; ++j) r += sm.cpart[j][0][threadIdx.x];
-        sm.r[threadIdx.x] = r;
-    }
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < DK * DV; idx += kBT) {
-        const int c = idx / DV, mm = idx % DV;
-        sm.S[c][mm] = fmaf(sm.k[c], sm.x[mm], fmaf(-sm.e[c], sm.r[mm], sm.al[c] * sm.S[c][mm]));
-    }
-    __syncthreads();
-}
-
-// State copies between global memory ([DK][DV], contiguous) and the padded shared array:
-// 16-byte global accesses, every load of a thread issued before its first store.
-template <int DK, int DV>
-__device__ void store_state(const Smem<DK, DV>& sm, float* dst) {
-    constexpr int N4 = DK * DV / 4 / kBT;
-#pragma unroll
-    for (int j = 0; j < N4; ++j) {
-        const int i4 = threadIdx.x + j * kBT, c = (4 * i4) / DV, m = (4 * i4) % DV;
-        reinterpret_cast<float4*>(dst)[i4] = make_float4(sm.S[c][m], sm.S[c][m + 1], sm.S[c][m + 2], sm.S[c][m + 3]);
-    }
-}
-template <int DK, int DV>
-__device__ void load_state(Smem<DK, DV>& sm, const float* src) {
-    constexpr int N4 = DK * DV / 4 / kBT;
-    float4 r[N4];
-#pragma unroll
-    for (int j = 0; j < N4; ++j)
-        r[j] = src ? reinterpret_cast<const float4*>(src)[threadIdx.x + j * kBT] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < N4; ++j) {
-        const int i4 = threadIdx.x + j * kBT, c = (4 * i4) / DV, m = (4 * i4) % DV;
-        sm.S[c][m] = r[j].x;
-        sm.S[c][m + 1] = r[j].y;
-        sm.S[c][m + 2] = r[j].z;
-        sm.S[c][m + 3] = r[j].w;
-    }
-}
-
-template <int DK, int DV, typename T>
-__global__ void __launch_bounds__(kBT, 1) chunk_bwd_kernel(const __grid_constant__ BwdParams bp) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    Smem<DK, DV>& sm = *reinterpret_cast<Smem<DK, DV>*>(smem_raw);
     const Params& p = bp.f;
     const int item = blockIdx.x;
     const int n = item / p.h_v, h = item % p.h_v, g = h / (p.h_v / p.h_qk);
     int t0, t1;
     seq_bounds(p, n, t0, t1);
-    const int nck = (t1 - t0 + kCk - 1) / kCk;
-    // this sequence's first checkpoint: the chunks of the sequences before it
-    int base = 0;
-    if (p.cu_seqlens) {
-        for (int j = 0; j < n; ++j) {
-            int a0, a1;
-            seq_bounds(p, j, a0, a1);
-            base += (a1 - a0 + kCk - 1) / kCk;
-        }
-    } else {
-        base = n * ((p.T_fixed + kCk - 1) / kCk);
-    }
-    const size_t SZ = (size_t)DK * DV;
-    float* ck = bp.ckpt + (size_t)base * p.h_v * SZ;
-    auto ckpt_of = [&](int c) { return ck + ((size_t)c * p.h_v + h) * SZ; };
-    float* scr = bp.scratch + (size_t)item * kCk * SZ;
-    const size_t soff = ((size_t)n * p.h_v + h) * SZ;
+    const int nsub = (t1 - t0 + kL - 1) / kL;
+    const size_t soff = ((size_t)n * p.h_v + h) * DK * DV;
+    const size_t slot0 = (size_t)n + t0 / kL;  // distinct per sub-chunk over all sequences
+    auto ckpt = [&](int s) { return bp.ckpt + ((slot0 + s) * p.h_v + h) * C::S4; };
+    auto scr = [&](int i) { return bp.scratch + ((size_t)item * (kL - 1) + i) * C::S4; };
 
-    // ---- forward: checkpoints at the start of every chunk
-    load_state(sm, p.S0 ? p.S0 + soff : nullptr);
-    __syncthreads();
-    for (int c = 0; c < nck; ++c) {
-        store_state(sm, ckpt_of(c));
-        const int te = min(t0 + (c + 1) * kCk, t1);
-        for (int t = t0 + c * kCk; t < te; ++t) {
-            load_token<DK, DV, T>(p, sm, (size_t)t, g, h, nullptr);
-            __syncthreads();
-            forward_token(sm);
-        }
-    }
+    float S[RJ][kMC], dS[RJ][kMC];
+    load_rowmajor<DK, DV>(S, p.S0 ? p.S0 + soff : nullptr, warp, lane);
+    load_rowmajor<DK, DV>(dS, bp.dS_T ? bp.dS_T + soff : nullptr, warp, lane);
 
-    // ---- backward
-    for (int idx = threadIdx.x; idx < DK * DV; idx += kBT)
-        sm.dS[idx / DV][idx % DV] = bp.dS_T ? bp.dS_T[soff + idx] : 0.f;
-    for (int c = nck - 1; c >= 0; --c) {
-        const int ts = t0 + c * kCk, te = min(ts + kCk, t1);
-        // the chunk's states: scr[i] = the state after token ts + i (i < te - ts - 1)
+    // Phases k = 0 .. nsub-2 are the checkpointing pass over sub-chunks 0 .. nsub-2; phases
+    // nsub-1 .. 2 nsub-2 are the backward over sub-chunks nsub-1 .. 0. Phase k's tokens are
+    // in token buffer k & 1, queued during phase k - 1.
+    const int K = nsub > 0 ? 2 * nsub - 1 : 0;
+    auto sub_of = [&](int k) { return k < nsub - 1 ? k : 2 * (nsub - 1) - k; };
+    auto queue = [&](int k) {
+        const int s = sub_of(k), ts = t0 + s * kL;
+        issue_tokens<DK, DV, T>(bp, tok + (k & 1) * kL * C::REC, ts, min(kL, t1 - ts), g, h, k >= nsub - 1);
+    };
+    auto next_phase = [&](int k) {
+        cp_async_wait_all();
         __syncthreads();
-        load_state(sm, ckpt_of(c));
-        __syncthreads();
-        for (int t = ts; t + 1 < te; ++t) {
-            load_token<DK, DV, T>(p, sm, (size_t)t, g, h, nullptr);
-            __syncthreads();
-            forward_token(sm);
-            store_state(sm, scr + (size_t)(t - ts) * SZ);
+        if (k + 1 < K) queue(k + 1);
+        cp_async_commit();
+    };
+    if (K > 0) queue(0);
+    cp_async_commit();
+    for (int k = 0; k + 1 < nsub; ++k) {
+        next_phase(k);
+        put_slice<DK>(ckpt(k), S, warp, lane);
+        const uint8_t* tb = tok + (k & 1) * kL * C::REC;
+        for (int i = 0; i < kL; ++i) fwd_step<DK, DV, T>(S, tb + i * C::REC, col, lane, warp);
+    }
+    if (nsub > 0) {
+        put_slice<DK>(ckpt(nsub - 1), S, warp, lane);
+        put_slice<DK>(spb + C::S4, S, warp, lane);  // the last sub-chunk's start state
+    }
+    int pb = 0;
+    for (int k = max(nsub - 1, 0); k < K; ++k) {
+        next_phase(k);
+        const int s = sub_of(k), ts = t0 + s * kL, len = min(kL, t1 - ts);
+        const uint8_t* tb = tok + (k & 1) * kL * C::REC;
+        // ---- backward over sub-chunk s: its start state (buffer 1) was put there before this
+        // loop or prefetched by the previous sub-chunk's last token; recompute the states
+        // after tokens ts .. ts + len - 2 into scratch, the last of them straight into the
+        // S_prev buffer of token ts + len - 1.
+        get_slice<DK>(S, spb + C::S4, warp, lane);
+        for (int i = 0; i + 1 < len; ++i) {
+            fwd_step<DK, DV, T>(S, tb + i * C::REC, col, lane, warp);
+            if (i + 2 < len) put_slice<DK>(scr(i), S, warp, lane);
         }
-        for (int t = te - 1; t >= ts; --t) {
-            __syncthreads();
-            load_state(sm, t == ts ? ckpt_of(c) : scr + (size_t)(t - ts - 1) * SZ);  // S_prev
-            load_token<DK, DV, T>(p, sm, (size_t)t, g, h, bp.dO);
-            __syncthreads();
-            // pass A: dS += q dO^T; column sums r = S'^T k, dx = dS^T k, dr = -dS^T e
+        put_slice<DK>(spb + ((len - 1) & 1) * C::S4, S, warp, lane);
+        // S_prev of token ts + i (i < len - 1): the checkpoint for i = 0, else scratch state i - 1
+        auto sprev = [&](int i) -> const float4* { return i == 0 ? ckpt(s) : scr(i - 1); };
+        for (int i = len - 1; i >= 0; --i) {
+            const uint8_t* rec = tb + i * C::REC;
+            const size_t t = (size_t)ts + i;
+            cp_async_wait_all();
+            float SP[RJ][kMC];
+            get_slice<DK>(SP, spb + (i & 1) * C::S4, warp, lane);
+            if (i > 0) copy_slice_async<DK>(spb + ((i - 1) & 1) * C::S4, sprev(i - 1), warp, lane);
+            else if (s > 0) copy_slice_async<DK>(spb + C::S4, ckpt(s - 1), warp, lane);
+            cp_async_commit();
+
+            const auto rv = row_vals<DK, DV, T>(rec, lane);
+            float dO[16];
+            ld16(reinterpret_cast<const float*>(rec + C::OFF_DO) + kMC * warp, dO);
+            // dS += q dO^T; column sums r = S'^T k, dx = dS^T k, dr = -dS^T e
+            float a[3][16];
+#pragma unroll
+            for (int mm = 0; mm < 16; ++mm) {
+                float ar = 0.f, ax = 0.f, ad = 0.f;
+#pragma unroll
+                for (int j = 0; j < RJ; ++j) {
+                    const float d = fmaf(rv.q[j], dO[mm], dS[j][mm]);
+                    dS[j][mm] = d;
+                    ar = fmaf(rv.al[j] * rv.k[j], SP[j][mm], ar);
+                    ax = fmaf(rv.k[j], d, ax);
+                    ad = fmaf(-rv.e[j], d, ad);
+                }
+                a[0][mm] = ar; a[1][mm] = ax; a[2][mm] = ad;
+            }
+            col_reduce<3>(a, lane);
+            __syncwarp();
+            if (!(lane & 1)) {
+                const int mc = lane >> 1, m = kMC * warp + mc;
+                col[mc] = a[0][0];
+                col[kMC + mc] = a[2][0];
+                const size_t tv = t * p.h_v + h;
+                bp.dw[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(rec + C::OFF_V)[m]);
+                bp.dv[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(rec + C::OFF_W)[m]);
+            }
+            __syncwarp();
+            float r[16], dr[16], x[16];
+            ld16(col, r);
+            ld16(col + kMC, dr);
             {
-                constexpr int CP = kBT / DV;
-                const int m = threadIdx.x % DV, part = threadIdx.x / DV;
-                const float dom = sm.dO[m];
-                float ar = 0.f, adx = 0.f, adr = 0.f;
-                for (int cc = part; cc < DK; cc += CP) {
-                    const float d = fmaf(sm.q[cc], dom, sm.dS[cc][m]);
-                    sm.dS[cc][m] = d;
-                    ar = fmaf(sm.al[cc] * sm.k[cc], sm.S[cc][m], ar);
-                    adx = fmaf(sm.k[cc], d, adx);
-                    adr = fmaf(-sm.e[cc], d, adr);
-                }
-                sm.cpart[part][0][m] = ar;
-                sm.cpart[part][1][m] = adx;
-                sm.cpart[part][2][m] = adr;
-                __syncthreads();
-                if (threadIdx.x < DV) {
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+                float v[16], w[16];
+                ld16(reinterpret_cast<const T*>(rec + C::OFF_V) + kMC * warp, v);
+                ld16(reinterpret_cast<const T*>(rec + C::OFF_W) + kMC * warp, w);
 #pragma unroll
-                    for (int j = 0; j < CP; ++j) {
-                        a0 += sm.cpart[j][0][threadIdx.x];
-                        a1 += sm.cpart[j][1][threadIdx.x];
-                        a2 += sm.cpart[j][2][threadIdx.x];
-                    }
-                    sm.r[threadIdx.x] = a0;
-                    sm.dx[threadIdx.x] = a1;
-                    sm.dr[threadIdx.x] = a2;
-                }
-                __syncthreads();
+                for (int mm = 0; mm < 16; ++mm) x[mm] = w[mm] * v[mm];
             }
-            // r . dO and x . dO (warps 0 and 1)
-            if (threadIdx.x < 64) {
-                const int wi = threadIdx.x / 32, l = threadIdx.x % 32;
-                float s = 0.f;
-                for (int m = l; m < DV; m += 32) s = fmaf(wi == 0 ? sm.r[m] : sm.x[m], sm.dO[m], s);
+            float rdo = 0.f, xdo = 0.f;
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-                if (l == 0) sm.dots[wi] = s;
+            for (int mm = 0; mm < 16; ++mm) {
+                rdo = fmaf(r[mm], dO[mm], rdo);
+                xdo = fmaf(x[mm], dO[mm], xdo);
             }
-            // pass B: row sums; dS <- Diag(alpha) (dS + k dr^T)
-            {
-                constexpr int RP = kBT / DK;
-                const int cc = threadIdx.x % DK, part = threadIdx.x / DK;
-                const float kc = sm.k[cc], alc = sm.al[cc];
-                float ade = 0.f, adk = 0.f, ada = 0.f, asd = 0.f;
-                for (int m = part; m < DV; m += RP) {
-                    const float d = sm.dS[cc][m], sp = sm.S[cc][m], drm = sm.dr[m];
-                    const float dsp = fmaf(kc, drm, d);
-                    ade = fmaf(-d, sm.r[m], ade);
-                    adk = fmaf(d, sm.x[m], fmaf(alc * sp, drm, adk));
-                    ada = fmaf(dsp, sp, ada);
-                    asd = fmaf(sp, sm.dO[m], asd);
-                    sm.dS[cc][m] = alc * dsp;
-                }
-                sm.rpart[part][0][cc] = ade;
-                sm.rpart[part][1][cc] = adk;
-                sm.rpart[part][2][cc] = ada;
-                sm.rpart[part][3][cc] = asd;
-                __syncthreads();
-                if (threadIdx.x < DK) {
-                    float de = 0.f, dk = 0.f, da = 0.f, sd = 0.f;
+            // row sums over the warp's columns; dS <- Diag(alpha) (dS + k dr^T)
+            float* pw = part + ((size_t)pb * C::NW + warp) * 4 * DK;
 #pragma unroll
-                    for (int j = 0; j < RP; ++j) {
-                        de += sm.rpart[j][0][cc];
-                        dk += sm.rpart[j][1][cc];
-                        da += sm.rpart[j][2][cc];
-                        sd += sm.rpart[j][3][cc];
-                    }
-                    const size_t tq = (size_t)t * p.h_qk + g, tv = (size_t)t * p.h_v + h;
-                    dk += de * sm.b[cc];
-                    const float dq = alc * sd - sm.e[cc] * sm.dots[0] + kc * sm.dots[1];
-                    if (bp.atomic_qk) {
-                        atomicAdd(bp.dq + tq * DK + cc, dq);
-                        atomicAdd(bp.dk + tq * DK + cc, dk);
-                    } else {
-                        bp.dq[tq * DK + cc] = dq;
-                        bp.dk[tq * DK + cc] = dk;
-                    }
-                    bp.db[tv * DK + cc] = de * kc;
-                    bp.dla[tv * DK + cc] = da * alc;
+            for (int j = 0; j < RJ; ++j) {
+                float pde = 0.f, pdk = 0.f, pdr = 0.f, pda = 0.f, psd = 0.f;
+#pragma unroll
+                for (int mm = 0; mm < 16; ++mm) {
+                    const float d = dS[j][mm], sp = SP[j][mm];
+                    const float dsp = fmaf(rv.k[j], dr[mm], d);
+                    pde = fmaf(d, r[mm], pde);
+                    pdk = fmaf(d, x[mm], pdk);
+                    pdr = fmaf(sp, dr[mm], pdr);
+                    pda = fmaf(dsp, sp, pda);
+                    psd = fmaf(sp, dO[mm], psd);
+                    dS[j][mm] = rv.al[j] * dsp;
                 }
-                if (threadIdx.x < DV) {
-                    const int m = threadIdx.x;
-                    const size_t tv = (size_t)t * p.h_v + h;
-                    bp.dw[tv * DV + m] = sm.dx[m] * sm.v[m];
-                    bp.dv[tv * DV + m] = sm.dx[m] * sm.w[m];
+                const int c = lane + 32 * j;
+                pw[c] = fmaf(rv.al[j], psd, fmaf(-rv.e[j], rdo, rv.k[j] * xdo));  // dq
+                pw[DK + c] = fmaf(rv.al[j], pdr, fmaf(-rv.b[j], pde, pdk));       // dk
+                pw[2 * DK + c] = -rv.k[j] * pde;                                   // db
+                pw[3 * DK + c] = rv.al[j] * pda;                                   // dlog_alpha
+            }
+            __syncthreads();
+            const float* pr = part + (size_t)pb * C::NW * 4 * DK;
+            for (int o = threadIdx.x; o < 4 * DK; o += C::NT) {
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < C::NW; ++w) sum += pr[w * 4 * DK + o];
+                const int which = o / DK, c = o - which * DK;
+                const size_t iq = (t * p.h_qk + g) * DK + c, iv = (t * p.h_v + h) * DK + c;
+                if (which == 0) {
+                    if (bp.atomic_qk) atomicAdd(bp.dq + iq, sum); else bp.dq[iq] = sum;
+                } else if (which == 1) {
+                    if (bp.atomic_qk) atomicAdd(bp.dk + iq, sum); else bp.dk[iq] = sum;
+                } else if (which == 2) {
+                    bp.db[iv] = sum;
+                } else {
+                    bp.dla[iv] = sum;
                 }
             }
+            pb ^= 1;
         }
     }
-    __syncthreads();
-    if (bp.dS0)
-        for (int idx = threadIdx.x; idx < DK * DV; idx += kBT) bp.dS0[soff + idx] = sm.dS[idx / DV][idx % DV];
+    cp_async_wait_all();
+    if (bp.dS0) {
+        float4* dst = reinterpret_cast<float4*>(bp.dS0 + soff);
+#pragma unroll
+        for (int j = 0; j < RJ; ++j)
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+                dst[gidx<DV>(warp, lane, j, qq)] =
+                    make_float4(dS[j][4 * qq], dS[j][4 * qq + 1], dS[j][4 * qq + 2], dS[j][4 * qq + 3]);
+    }
 }
 
 template <int DK, int DV, typename T>
 cudaError_t launch_bwd_t(const BwdParams& bp, cudaStream_t s) {
-    const size_t smem = sizeof(Smem<DK, DV>);
+    using C = Cfg<DK, DV, T>;
+    static_assert(C::SMEM <= 227 * 1024, "backward shared memory");
     cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<DK, DV, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+                                         C::SMEM);
     if (e != cudaSuccess) return e;
-    chunk_bwd_kernel<DK, DV, T><<<bp.f.n_seq * bp.f.h_v, kBT, smem, s>>>(bp);
+    chunk_bwd_kernel<DK, DV, T><<<bp.f.n_seq * bp.f.h_v, C::NT, C::SMEM, s>>>(bp);
     return cudaGetLastError();
 }
 
@@ -294,12 +444,14 @@ cudaError_t launch_bwd_d(const BwdParams& bp, cudaStream_t s) {
     return bp.f.dv == 128 ? launch_bwd_t<64, 128, T>(bp, s) : launch_bwd_t<64, 64, T>(bp, s);
 }
 
+// Checkpoint slots: n + t0 / kL + s is below this for every sub-chunk s of every sequence n.
+size_t ckpt_slots(int T_total, int n_seq) { return (size_t)(T_total + kL - 1) / kL + (size_t)n_seq; }
+
 }  // namespace
 
 size_t bwd_workspace_bytes(const gdn2_shape* sh) {
     const size_t SZ = (size_t)sh->dk * sh->dv * sizeof(float);
-    const size_t chunks = (size_t)(sh->T_total + kCk - 1) / kCk + (size_t)sh->n_seq;  // >= sum of per-sequence chunks
-    return chunks * sh->h_v * SZ + (size_t)sh->n_seq * sh->h_v * kCk * SZ;
+    return ckpt_slots(sh->T_total, sh->n_seq) * sh->h_v * SZ + (size_t)sh->n_seq * sh->h_v * (kL - 1) * SZ;
 }
 
 cudaError_t launch_bwd(const Params& p, gdn2_dtype dt, const float* dO, const float* dS_T, float* dq, float* dk,
@@ -308,10 +460,9 @@ cudaError_t launch_bwd(const Params& p, gdn2_dtype dt, const float* dO, const fl
     bp.f = p;
     bp.dO = dO; bp.dS_T = dS_T;
     bp.dq = dq; bp.dk = dk; bp.dv = dv; bp.dla = dla; bp.db = db; bp.dw = dw; bp.dS0 = dS0;
-    const size_t SZ = (size_t)p.dk * p.dv;
-    const size_t chunks = (size_t)(p.T_total + kCk - 1) / kCk + (size_t)p.n_seq;
-    bp.ckpt = static_cast<float*>(workspace);
-    bp.scratch = bp.ckpt + chunks * p.h_v * SZ;
+    const size_t S4 = (size_t)p.dk * p.dv / 4;
+    bp.ckpt = static_cast<float4*>(workspace);
+    bp.scratch = bp.ckpt + ckpt_slots(p.T_total, p.n_seq) * p.h_v * S4;
     bp.atomic_qk = p.h_v != p.h_qk;
     if (bp.atomic_qk) {
         const size_t qk_bytes = (size_t)p.T_total * p.h_qk * p.dk * sizeof(float);

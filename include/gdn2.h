@@ -183,10 +183,11 @@ GDN2_API gdn2_status gdn2_chunk_fwd_prologue(const gdn2_shape* shape,
  *   dv, dw [T_total, h_v, dv];  dlog_alpha, db [T_total, h_v, dk]
  *   dS0 (nullable) [n_seq, h_v, dk, dv].
  * The pages describe the forward recurrence only (they state the model was trained, which
- * needs these); the derivation is the chain rule through the per-token update. This first
- * form runs one CTA per (sequence, value head), sequentially: a forward pass storing the
- * state at every 64th token, then, chunk by chunk from the end, the chunk's states are
- * recomputed into a scratch area and its tokens walked backwards.
+ * needs these); the derivation is the chain rule through the per-token update, in fp32.
+ * One CTA runs per (sequence, value head), each warp owning 16 value columns of the state
+ * in registers: a forward pass stores the state at every 8th token, then, from the end, each
+ * 8-token sub-chunk's states are recomputed into a scratch area and its tokens walked
+ * backwards.
  * workspace: device memory of gdn2_chunk_bwd_workspace_size(shape) bytes, 256-byte
  * aligned (required). With h_v > h_qk, dq and dk are zeroed on the stream and accumulated
  * with atomics (the order of those additions varies from run to run).
