@@ -33,6 +33,11 @@ sys.path.insert(0, ROOT)
 
 PREFILL = "prefill_b8_h16_t4096"
 DECODE = "decode_256seq_h32"
+GROUPED = "grouped_b2_qk16_v32_t32768"
+GROUPED_TIMED_STEPS = 5
+# fp32 SIMT peak for the backward's per-token adjoint: 148 SMs x 128 fp32 lanes x 2 flop
+# (one FMA) per clock at the 1965 MHz maximum SM clock
+FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 SERVING_TOKENS = 4  # tokens per sequence in one serving-decode step (a verify step)
 PROLOGUE_TIMED_STEPS = 10
 BACKWARD_TIMED_STEPS = 3
@@ -162,6 +167,15 @@ def backward_bytes(wl, lengths) -> int:
     writes = wl.h_qk * 2 * wl.dk * 4 + wl.h_v * (2 * wl.dv * 4 + 2 * wl.dk * 4)
     state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
     return T * (reads + writes) + state * 2
+
+
+def backward_flops(wl, lengths) -> int:
+    """Algorithmic fp32 flops of one backward by the per-token adjoint: per token, value
+    head and state element, 7 to regenerate S_prev (r: one FMA; update: a multiply and two
+    FMAs) and 21 for the adjoint (ten FMAs: dS += q dO, r, dx, dr, dS', de, dk (two),
+    dalpha, dq; one multiply: dS <- alpha dS'). The kernel's second forward pass (the
+    recompute from checkpoints) is not counted."""
+    return int(sum(lengths)) * wl.h_v * wl.dk * wl.dv * 28
 
 
 def serving_bytes(wl, n_tok: int) -> int:
@@ -366,13 +380,49 @@ def main():
     bms = max_over_ranks(e0.elapsed_time(e1) / BACKWARD_TIMED_STEPS, world)
     bbytes = backward_bytes(wl, d["lengths"])
     bach = bbytes / (bms / 1000.0) / 1e9
+    bflops = backward_flops(wl, d["lengths"])
+    btf = bflops / (bms / 1000.0) / 1e12
     backward = {"metric": "GDN-2 backward tokens/s", "value": world * T_all / (bms / 1000.0), "unit": "tokens/s",
                 "ms_per_step": bms, "steps": BACKWARD_TIMED_STEPS,
                 "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (per-token adjoint, fp32, column slices per warp)"},
-                "roofline": {"bound": "hbm", "achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
-                             "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
-                             "algorithmic_bytes_per_launch": bbytes}}
+                "roofline": {"bound": "alu", "achieved": btf, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
+                             "frac": btf / FP32_SIMT_TFLOPS, "traffic": None,
+                             "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
+                             "algorithmic_flops_per_launch": bflops,
+                             "hbm": {"achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
+                                     "algorithmic_bytes_per_launch": bbytes}}}
     del dO_b, ws_b
+
+    # ---------------- grouped heads: 16 query/key heads shared by 32 value heads, with S0
+    gwl = W.WORKLOADS[GROUPED]
+    gd = W.prefill_inputs(gwl, dev)
+    g_o = torch.empty(gd["v"].shape, dtype=torch.float32, device=dev)
+    g_S = torch.empty_like(gd["S0"])
+    gstep = lambda: G.gdn2_chunk_fwd(gd["q"], gd["k"], gd["v"], gd["log_alpha"], gd["b"], gd["w"], S0=gd["S0"],
+                                     n_seq=gd["n_seq"], o=g_o, S_T=g_S, stream=stream)
+    for _ in range(3):
+        gstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(GROUPED_TIMED_STEPS):
+        gstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    gms = max_over_ranks(e0.elapsed_time(e1) / GROUPED_TIMED_STEPS, world)
+    g_T = int(sum(gd["lengths"]))
+    gbytes = prefill_bytes(gwl, gd["lengths"])
+    gach = gbytes / (gms / 1000.0) / 1e9
+    grouped = {"metric": "GDN-2 chunk-fwd tokens/s, grouped heads", "value": world * g_T / (gms / 1000.0),
+               "unit": "tokens/s", "ms_per_step": gms, "steps": GROUPED_TIMED_STEPS,
+               "config": {"workload": GROUPED, "global_batch": gwl.n_seq, "seq_len": gwl.T, "qk_heads": gwl.h_qk,
+                          "v_heads": gwl.h_v, "dk": gwl.dk, "dv": gwl.dv,
+                          "bytes": "q, k counted once per query/key head"},
+               "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm, "unit": "GB/s", "frac": gach / hbm,
+                            "traffic": recorded_traffic("chunk_tc_grouped_b2_qk16_v32.md",
+                                                        "gated_delta_rule_160_b200/csrc/chunk_tc.cu"),
+                            "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": gbytes}}
+    del gd, g_o, g_S
 
     # ---------------- decode (the second metric)
     dwl = W.WORKLOADS[DECODE]
@@ -494,6 +544,7 @@ def main():
             "serving_decode": serving,
             "prefill_prologue": prologue,
             "backward": backward,
+            "grouped": grouped,
             "e2e": e2e,
             "cpu_baseline": base,
             "clocks": clocks.summary(),

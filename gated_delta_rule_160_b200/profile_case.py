@@ -2,11 +2,16 @@
 
     python -m gated_delta_rule_160_b200.profile_case --kernel chunk --n-seq 2 --iters 3
     python -m gated_delta_rule_160_b200.profile_case --kernel decode --n-seq 64 --iters 3
+    python -m gated_delta_rule_160_b200.profile_case --kernel bwd --n-seq 2 --T 1024 --iters 2
+    python -m gated_delta_rule_160_b200.profile_case --kernel grouped --n-seq 2 --T 8192 --iters 3
 
 ``chunk`` runs gdn2_chunk_fwd on the first ``n-seq`` sequences of the 16-head, T=4096,
-d=128 bf16 prefill workload (2 sequences: 268 MB of inputs, larger than L2); ``decode``
-runs gdn2_decode_step on ``n-seq`` sequences of the 32-head decode workload. Each kernel
-is launched ``iters`` times; profile the last launches (ncu -s / -c).
+d=128 bf16 prefill workload (2 sequences: 268 MB of inputs, larger than L2; ``T`` cuts them); ``decode``
+runs gdn2_decode_step on ``n-seq`` sequences of the 32-head decode workload; ``bwd`` runs
+gdn2_chunk_bwd (gradients of sum(o * dO)) on the prefill workload's first ``n-seq``
+sequences; ``grouped`` runs gdn2_chunk_fwd on the grouped-head workload (16 query/key heads
+shared by 32 value heads, with an initial state), its sequences cut to ``T`` tokens. Each
+kernel is launched ``iters`` times; profile the last launches (ncu -s / -c).
 """
 import argparse
 
@@ -18,17 +23,34 @@ from gated_delta_rule_160_b200 import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["chunk", "decode"], default="chunk")
+    ap.add_argument("--kernel", choices=["chunk", "decode", "bwd", "grouped"], default="chunk")
     ap.add_argument("--n-seq", type=int, default=2)
+    ap.add_argument("--T", type=int, default=None, help="tokens per sequence (chunk, bwd, grouped)")
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
     G.load_library()
-    if a.kernel == "chunk":
+    if a.kernel in ("chunk", "bwd"):
         wl = W.WORKLOADS["prefill_b8_h16_t4096"]
-        d = W.prefill_inputs(wl, "cuda", n_seq=a.n_seq)
+        d = W.prefill_inputs(wl, "cuda", n_seq=a.n_seq, T=a.T)
         o = torch.empty(d["v"].shape, dtype=torch.float32, device="cuda")
+        if a.kernel == "chunk":
+            for _ in range(a.iters):
+                G.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], n_seq=a.n_seq, o=o)
+        else:
+            dO = torch.randn(o.shape, generator=torch.Generator(device="cuda").manual_seed(wl.seed + 29),
+                             device="cuda")
+            ws = None
+            for _ in range(a.iters):
+                G.gdn2_chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], dO, n_seq=a.n_seq,
+                                 want_dS0=False, workspace=ws)
+    elif a.kernel == "grouped":
+        wl = W.WORKLOADS["grouped_b2_qk16_v32_t32768"]
+        d = W.prefill_inputs(wl, "cuda", n_seq=a.n_seq, T=a.T)
+        o = torch.empty(d["v"].shape, dtype=torch.float32, device="cuda")
+        S_T = torch.empty_like(d["S0"])
         for _ in range(a.iters):
-            G.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], n_seq=a.n_seq, o=o)
+            G.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=d["S0"], n_seq=a.n_seq,
+                             o=o, S_T=S_T)
     else:
         wl = W.WORKLOADS["decode_256seq_h32"]
         S = W.decode_state(wl, "cuda", n_seq=a.n_seq)
