@@ -384,7 +384,7 @@ def main():
     btf = bflops / (bms / 1000.0) / 1e12
     backward = {"metric": "GDN-2 backward tokens/s", "value": world * T_all / (bms / 1000.0), "unit": "tokens/s",
                 "ms_per_step": bms, "steps": BACKWARD_TIMED_STEPS,
-                "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (per-token adjoint, fp32, column slices per warp)"},
+                "config": {"workload": f"{PREFILL}, gradients of sum(o * dO) (per-token adjoint, fp32, 8 value columns per warp)"},
                 "roofline": {"bound": "alu", "achieved": btf, "peak": FP32_SIMT_TFLOPS, "unit": "TFLOP/s",
                              "frac": btf / FP32_SIMT_TFLOPS, "traffic": None,
                              "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",

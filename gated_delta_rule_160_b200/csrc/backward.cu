@@ -12,28 +12,32 @@
 //
 // Every value column of the state evolves on its own: the forward update and the adjoint of
 // column m read only column m and the token's key-side vectors. So one CTA per (sequence,
-// value head) gives each warp 16 value columns and keeps that dk x 16 slice of S_prev and of
-// dS in registers (lane l holds key rows l, l + 32, ...). Column sums (r, dx, dr) are a warp
-// reduction; the per-row gradients (dq, dk, db, dlog_alpha) are sums over all columns, so each
-// warp writes its partial row sums to shared memory and, after one barrier per token, the CTA
-// adds the warps' partials and writes the outputs.
+// value head) gives each warp 8 value columns and keeps that dk x 8 slice of S_prev and of
+// dS in registers (lane l holds key rows l, l + 32, ...): 16 warps for dv = 128, four per
+// scheduler. Column sums (r, dx, dr) are a warp reduction; the per-row gradients (dq, dk,
+// db, dlog_alpha) are sums over all columns, so each warp writes its partial row sums to
+// shared memory and, after one barrier per token, the CTA adds the warps' partials and
+// writes the outputs.
 //
 // Forward, then backward, over sub-chunks of kL tokens: a first pass stores the state at the
 // start of every sub-chunk (checkpoints); then, from the last sub-chunk, the sub-chunk's states
 // are recomputed from its checkpoint into a per-CTA scratch area (small enough to stay in L2)
 // and its tokens are walked backwards. Each thread stores and reloads only its own slice of a
 // state, in its own register order, so these copies need no synchronisation; the next token's
-// S_prev is prefetched with cp.async into a per-thread double buffer while the current one is
-// processed. Token inputs are staged in shared memory a sub-chunk at a time, double-buffered.
-// A query/key head's dq, dk sum over the value heads that read it: with groups of several
-// value heads they are accumulated with atomics into outputs the host zeroed first.
+// S_prev is fetched with cp.async into shared memory while the current token is processed.
+// A sub-chunk's inputs are staged in shared memory with cp.async (double-buffered) and then
+// turned, once, into the fp32 operands every pass reads: alpha k, b k, k, alpha, q, b per key
+// row and w v, dO per value column. A query/key head's dq, dk sum over the value heads that
+// read it: with groups of several value heads they are accumulated with atomics into outputs
+// the host zeroed first.
 #include "internal.cuh"
 
 namespace gdn2 {
 namespace {
 
 constexpr int kL = 8;        // tokens per sub-chunk (checkpoint interval)
-constexpr int kMC = 16;      // value columns per warp
+constexpr int kMC = 8;       // value columns per warp
+constexpr int kQ = kMC / 4;  // float4 per key row of a warp's slice
 
 struct BwdParams {
     Params f;                // the forward's arguments
@@ -52,36 +56,24 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// 16 consecutive values (16-byte aligned) as fp32; a warp reading one address broadcasts.
-__device__ __forceinline__ void ld16(const float* p, float (&o)[16]) {
+// kMC consecutive fp32 values (16-byte aligned); a warp reading one address broadcasts.
+__device__ __forceinline__ void ldc(const float* p, float (&o)[kMC]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kQ; ++i) {
         const float4 u = reinterpret_cast<const float4*>(p)[i];
         o[4 * i] = u.x; o[4 * i + 1] = u.y; o[4 * i + 2] = u.z; o[4 * i + 3] = u.w;
     }
 }
-__device__ __forceinline__ void ld16(const __nv_bfloat16* p, float (&o)[16]) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const uint4 u = reinterpret_cast<const uint4*>(p)[i];
-        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[j]));
-            o[8 * i + 2 * j] = f.x;
-            o[8 * i + 2 * j + 1] = f.y;
-        }
-    }
-}
 
-// Sums of a[v][0..15] over the warp's 32 lanes, NV vectors at once: each step hands half of
-// the remaining columns to the partner lane, so 8 + 4 + 2 + 1 + 1 shuffles per vector leave
-// in a[v][0] the full sum of column (lane >> 1).
+// Sums of a[v][0..7] over the warp's 32 lanes, NV vectors at once: each of the first three
+// steps hands half of the remaining columns to the partner lane (4 + 2 + 1 shuffles), two
+// more add the partners that hold the same column, leaving in a[v][0] the full sum of
+// column (lane >> 2).
 template <int NV>
-__device__ __forceinline__ void col_reduce(float (&a)[NV][16], int lane) {
+__device__ __forceinline__ void col_reduce(float (&a)[NV][kMC], int lane) {
 #pragma unroll
-    for (int st = 0; st < 4; ++st) {
-        const int half = 8 >> st, xm = 16 >> st;
+    for (int st = 0; st < 3; ++st) {
+        const int half = 4 >> st, xm = 16 >> st;
         const bool up = lane & xm;
 #pragma unroll
         for (int v = 0; v < NV; ++v)
@@ -93,29 +85,37 @@ __device__ __forceinline__ void col_reduce(float (&a)[NV][16], int lane) {
             }
     }
 #pragma unroll
-    for (int v = 0; v < NV; ++v) a[v][0] += __shfl_xor_sync(0xffffffffu, a[v][0], 1);
+    for (int v = 0; v < NV; ++v) {
+        a[v][0] += __shfl_xor_sync(0xffffffffu, a[v][0], 2);
+        a[v][0] += __shfl_xor_sync(0xffffffffu, a[v][0], 1);
+    }
 }
 
 template <int DK, int DV, typename T>
 struct Cfg {
     static constexpr int NW = DV / kMC, NT = 32 * NW, RJ = DK / 32;
     static constexpr int ES = sizeof(T);
-    // one token's inputs in shared memory: k, q, b, v, w (dtype), log_alpha, dO (fp32)
+    // one token's raw inputs in shared memory: k, q, b, v, w (dtype), log_alpha, dO (fp32)
     static constexpr int OFF_K = 0, OFF_Q = DK * ES, OFF_B = 2 * DK * ES, OFF_V = 3 * DK * ES;
     static constexpr int OFF_W = OFF_V + DV * ES, OFF_LA = OFF_W + DV * ES, OFF_DO = OFF_LA + 4 * DK;
     static constexpr int REC = OFF_DO + 4 * DV;
     static constexpr int CK = DK * ES / 16, CV = DV * ES / 16, CLA = DK / 4, CDO = DV / 4;
     static constexpr int CPT = 3 * CK + 2 * CV + CLA + CDO;  // 16-byte pieces per token
+    // one token's prepared fp32 operands: per key row {alpha k, b k, k, alpha} and {q, b};
+    // per value column w v and dO
+    static constexpr int PR_A = 0, PR_B = 16 * DK, PR_X = 24 * DK, PR_DO = PR_X + 4 * DV;
+    static constexpr int PREC = PR_DO + 4 * DV;
     static constexpr int S4 = DK * DV / 4;                   // float4 per state
     // shared memory (bytes)
-    static constexpr int SM_TOK = 0;                              // [2][kL][REC]
-    static constexpr int SM_SP = SM_TOK + 2 * kL * REC;           // [2][S4] float4: S_prev
-    static constexpr int SM_PART = SM_SP + 2 * S4 * 16;           // [2][NW][4][DK] f32: row partials
-    static constexpr int SM_COL = SM_PART + 2 * NW * 4 * DK * 4;  // [NW][2][16] f32: r, dr
+    static constexpr int SM_TOK = 0;                              // [2][kL][REC] raw inputs
+    static constexpr int SM_PREP = SM_TOK + 2 * kL * REC;         // [kL][PREC] prepared operands
+    static constexpr int SM_SP = SM_PREP + kL * PREC;             // [S4] float4: S_prev
+    static constexpr int SM_PART = SM_SP + S4 * 16;               // [2][NW][4][DK] f32: row partials
+    static constexpr int SM_COL = SM_PART + 2 * NW * 4 * DK * 4;  // [NW][2][kMC] f32: r, dr
     static constexpr int SMEM = SM_COL + NW * 2 * kMC * 4;
 };
 
-// Queue (cp.async) the inputs of tokens [ts, ts + len) into a token buffer.
+// Queue (cp.async) the raw inputs of tokens [ts, ts + len) into a token buffer.
 template <int DK, int DV, typename T>
 __device__ void issue_tokens(const BwdParams& bp, uint8_t* dst, int ts, int len, int g, int h, bool with_dO) {
     using C = Cfg<DK, DV, T>;
@@ -142,71 +142,73 @@ __device__ void issue_tokens(const BwdParams& bp, uint8_t* dst, int ts, int len,
     }
 }
 
-// Key-side values of a token for this lane's rows.
-template <int RJ>
-struct RowVals {
-    float k[RJ], q[RJ], al[RJ], b[RJ], e[RJ];
-};
+// Raw inputs of len tokens -> their prepared fp32 operands (one exp per key row and token).
 template <int DK, int DV, typename T>
-__device__ __forceinline__ RowVals<DK / 32> row_vals(const uint8_t* rec, int lane) {
+__device__ void prepare(const uint8_t* raw, uint8_t* prep, int len, bool with_dO) {
     using C = Cfg<DK, DV, T>;
-    RowVals<DK / 32> rv;
-    const T* kt = reinterpret_cast<const T*>(rec + C::OFF_K);
-    const T* qt = reinterpret_cast<const T*>(rec + C::OFF_Q);
-    const T* bt = reinterpret_cast<const T*>(rec + C::OFF_B);
-    const float* lat = reinterpret_cast<const float*>(rec + C::OFF_LA);
-#pragma unroll
-    for (int j = 0; j < C::RJ; ++j) {
-        const int c = lane + 32 * j;
-        rv.k[j] = to_f32(kt[c]);
-        rv.q[j] = to_f32(qt[c]);
-        rv.b[j] = to_f32(bt[c]);
-        rv.al[j] = expf(lat[c]);
-        rv.e[j] = rv.b[j] * rv.k[j];
+    for (int u = threadIdx.x; u < len * (DK + DV); u += C::NT) {
+        const int i = u / (DK + DV), c = u - i * (DK + DV);
+        const uint8_t* rec = raw + i * C::REC;
+        uint8_t* pr = prep + i * C::PREC;
+        if (c < DK) {
+            const float k = to_f32(reinterpret_cast<const T*>(rec + C::OFF_K)[c]);
+            const float q = to_f32(reinterpret_cast<const T*>(rec + C::OFF_Q)[c]);
+            const float b = to_f32(reinterpret_cast<const T*>(rec + C::OFF_B)[c]);
+            const float al = expf(reinterpret_cast<const float*>(rec + C::OFF_LA)[c]);
+            reinterpret_cast<float4*>(pr + C::PR_A)[c] = make_float4(al * k, b * k, k, al);
+            reinterpret_cast<float2*>(pr + C::PR_B)[c] = make_float2(q, b);
+        } else {
+            const int m = c - DK;
+            const float v = to_f32(reinterpret_cast<const T*>(rec + C::OFF_V)[m]);
+            const float w = to_f32(reinterpret_cast<const T*>(rec + C::OFF_W)[m]);
+            reinterpret_cast<float*>(pr + C::PR_X)[m] = w * v;
+            reinterpret_cast<float*>(pr + C::PR_DO)[m] =
+                with_dO ? reinterpret_cast<const float*>(rec + C::OFF_DO)[m] : 0.f;
+        }
     }
-    return rv;
 }
 
-// One forward token on this thread's slice S (key rows lane + 32 j, the warp's 16 columns).
+// One forward token on this thread's slice S (key rows lane + 32 j, the warp's kMC columns).
 template <int DK, int DV, typename T>
-__device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t* rec, float* col, int lane,
+__device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t* pr, float* col, int lane,
                                          int warp) {
     using C = Cfg<DK, DV, T>;
-    const auto rv = row_vals<DK, DV, T>(rec, lane);
-    float a[1][16];
+    const float4* A = reinterpret_cast<const float4*>(pr + C::PR_A);
+    float a[1][kMC];
 #pragma unroll
-    for (int mm = 0; mm < 16; ++mm) {
-        float s = 0.f;
+    for (int mm = 0; mm < kMC; ++mm) a[0][mm] = 0.f;
 #pragma unroll
-        for (int j = 0; j < C::RJ; ++j) s = fmaf(rv.al[j] * rv.k[j], S[j][mm], s);
-        a[0][mm] = s;
+    for (int j = 0; j < C::RJ; ++j) {
+        const float ak = A[lane + 32 * j].x;
+#pragma unroll
+        for (int mm = 0; mm < kMC; ++mm) a[0][mm] = fmaf(ak, S[j][mm], a[0][mm]);
     }
     col_reduce<1>(a, lane);
     __syncwarp();
-    if (!(lane & 1)) col[lane >> 1] = a[0][0];
+    if (!(lane & 3)) col[lane >> 2] = a[0][0];
     __syncwarp();
-    float r[16], v[16], w[16];
-    ld16(col, r);
-    ld16(reinterpret_cast<const T*>(rec + C::OFF_V) + kMC * warp, v);
-    ld16(reinterpret_cast<const T*>(rec + C::OFF_W) + kMC * warp, w);
+    float r[kMC], x[kMC];
+    ldc(col, r);
+    ldc(reinterpret_cast<const float*>(pr + C::PR_X) + kMC * warp, x);
 #pragma unroll
-    for (int j = 0; j < C::RJ; ++j)
+    for (int j = 0; j < C::RJ; ++j) {
+        const float4 rw = A[lane + 32 * j];  // alpha k, e, k, alpha
 #pragma unroll
-        for (int mm = 0; mm < 16; ++mm)
-            S[j][mm] = fmaf(rv.k[j], w[mm] * v[mm], fmaf(-rv.e[j], r[mm], rv.al[j] * S[j][mm]));
+        for (int mm = 0; mm < kMC; ++mm) S[j][mm] = fmaf(rw.z, x[mm], fmaf(-rw.y, r[mm], rw.w * S[j][mm]));
+    }
 }
 
 // A thread's slice of a state in its own order: float4 index of (row group j, column quad qq).
 template <int DK>
 __device__ __forceinline__ int sidx(int warp, int lane, int j, int qq) {
-    return warp * (DK / 32) * 128 + (j * 4 + qq) * 32 + lane;
+    return warp * (DK / 32) * kQ * 32 + (j * kQ + qq) * 32 + lane;
 }
 template <int DK>
 __device__ __forceinline__ void put_slice(float4* dst, const float (&S)[DK / 32][kMC], int warp, int lane) {
 #pragma unroll
     for (int j = 0; j < DK / 32; ++j)
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
+        for (int qq = 0; qq < kQ; ++qq)
             dst[sidx<DK>(warp, lane, j, qq)] =
                 make_float4(S[j][4 * qq], S[j][4 * qq + 1], S[j][4 * qq + 2], S[j][4 * qq + 3]);
 }
@@ -215,7 +217,7 @@ __device__ __forceinline__ void get_slice(float (&S)[DK / 32][kMC], const float4
 #pragma unroll
     for (int j = 0; j < DK / 32; ++j)
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < kQ; ++qq) {
             const float4 u = src[sidx<DK>(warp, lane, j, qq)];
             S[j][4 * qq] = u.x; S[j][4 * qq + 1] = u.y; S[j][4 * qq + 2] = u.z; S[j][4 * qq + 3] = u.w;
         }
@@ -225,7 +227,7 @@ __device__ __forceinline__ void copy_slice_async(float4* dst, const float4* src,
 #pragma unroll
     for (int j = 0; j < DK / 32; ++j)
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < kQ; ++qq) {
             const int i = sidx<DK>(warp, lane, j, qq);
             cp_async16(dst + i, src + i);
         }
@@ -240,7 +242,7 @@ __device__ __forceinline__ void load_rowmajor(float (&S)[DK / 32][kMC], const fl
 #pragma unroll
     for (int j = 0; j < DK / 32; ++j)
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < kQ; ++qq) {
             const float4 u = src ? reinterpret_cast<const float4*>(src)[gidx<DV>(warp, lane, j, qq)]
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             S[j][4 * qq] = u.x; S[j][4 * qq + 1] = u.y; S[j][4 * qq + 2] = u.z; S[j][4 * qq + 3] = u.w;
@@ -253,6 +255,7 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
     constexpr int RJ = C::RJ;
     extern __shared__ __align__(16) uint8_t smem[];
     uint8_t* tok = smem + C::SM_TOK;
+    uint8_t* prep = smem + C::SM_PREP;
     float4* spb = reinterpret_cast<float4*>(smem + C::SM_SP);
     float* part = reinterpret_cast<float*>(smem + C::SM_PART);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -269,106 +272,106 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
     auto ckpt = [&](int s) { return bp.ckpt + ((slot0 + s) * p.h_v + h) * C::S4; };
     auto scr = [&](int i) { return bp.scratch + ((size_t)item * (kL - 1) + i) * C::S4; };
 
-    float S[RJ][kMC], dS[RJ][kMC];
+    float S[RJ][kMC];
     load_rowmajor<DK, DV>(S, p.S0 ? p.S0 + soff : nullptr, warp, lane);
-    load_rowmajor<DK, DV>(dS, bp.dS_T ? bp.dS_T + soff : nullptr, warp, lane);
 
     // Phases k = 0 .. nsub-2 are the checkpointing pass over sub-chunks 0 .. nsub-2; phases
-    // nsub-1 .. 2 nsub-2 are the backward over sub-chunks nsub-1 .. 0. Phase k's tokens are
-    // in token buffer k & 1, queued during phase k - 1.
+    // nsub-1 .. 2 nsub-2 are the backward over sub-chunks nsub-1 .. 0. Phase k's raw inputs
+    // are in token buffer k & 1, queued during phase k - 1.
     const int K = nsub > 0 ? 2 * nsub - 1 : 0;
     auto sub_of = [&](int k) { return k < nsub - 1 ? k : 2 * (nsub - 1) - k; };
     auto queue = [&](int k) {
         const int s = sub_of(k), ts = t0 + s * kL;
         issue_tokens<DK, DV, T>(bp, tok + (k & 1) * kL * C::REC, ts, min(kL, t1 - ts), g, h, k >= nsub - 1);
     };
-    auto next_phase = [&](int k) {
+    // wait for phase k's inputs, queue phase k + 1's, prepare phase k's operands
+    auto start_phase = [&](int k, int len, bool with_dO) {
         cp_async_wait_all();
         __syncthreads();
         if (k + 1 < K) queue(k + 1);
         cp_async_commit();
+        prepare<DK, DV, T>(tok + (k & 1) * kL * C::REC, prep, len, with_dO);
+        __syncthreads();
     };
     if (K > 0) queue(0);
     cp_async_commit();
     for (int k = 0; k + 1 < nsub; ++k) {
-        next_phase(k);
+        start_phase(k, kL, false);
         put_slice<DK>(ckpt(k), S, warp, lane);
-        const uint8_t* tb = tok + (k & 1) * kL * C::REC;
-        for (int i = 0; i < kL; ++i) fwd_step<DK, DV, T>(S, tb + i * C::REC, col, lane, warp);
+        for (int i = 0; i < kL; ++i) fwd_step<DK, DV, T>(S, prep + i * C::PREC, col, lane, warp);
     }
     if (nsub > 0) {
         put_slice<DK>(ckpt(nsub - 1), S, warp, lane);
-        put_slice<DK>(spb + C::S4, S, warp, lane);  // the last sub-chunk's start state
+        put_slice<DK>(spb, S, warp, lane);  // the last sub-chunk's start state
     }
+    float dS[RJ][kMC];
+    load_rowmajor<DK, DV>(dS, bp.dS_T ? bp.dS_T + soff : nullptr, warp, lane);
     int pb = 0;
     for (int k = max(nsub - 1, 0); k < K; ++k) {
-        next_phase(k);
         const int s = sub_of(k), ts = t0 + s * kL, len = min(kL, t1 - ts);
+        start_phase(k, len, true);
         const uint8_t* tb = tok + (k & 1) * kL * C::REC;
-        // ---- backward over sub-chunk s: its start state (buffer 1) was put there before this
-        // loop or prefetched by the previous sub-chunk's last token; recompute the states
-        // after tokens ts .. ts + len - 2 into scratch, the last of them straight into the
-        // S_prev buffer of token ts + len - 1.
-        get_slice<DK>(S, spb + C::S4, warp, lane);
+        // ---- backward over sub-chunk s: its start state (in the S_prev buffer: put there
+        // before this loop or fetched by the previous sub-chunk's last token); recompute the
+        // states after tokens ts .. ts + len - 2 into scratch, the last of them straight
+        // into the S_prev buffer for token ts + len - 1.
+        get_slice<DK>(S, spb, warp, lane);
         for (int i = 0; i + 1 < len; ++i) {
-            fwd_step<DK, DV, T>(S, tb + i * C::REC, col, lane, warp);
+            fwd_step<DK, DV, T>(S, prep + i * C::PREC, col, lane, warp);
             if (i + 2 < len) put_slice<DK>(scr(i), S, warp, lane);
         }
-        put_slice<DK>(spb + ((len - 1) & 1) * C::S4, S, warp, lane);
+        put_slice<DK>(spb, S, warp, lane);
         // S_prev of token ts + i (i < len - 1): the checkpoint for i = 0, else scratch state i - 1
         auto sprev = [&](int i) -> const float4* { return i == 0 ? ckpt(s) : scr(i - 1); };
         for (int i = len - 1; i >= 0; --i) {
-            const uint8_t* rec = tb + i * C::REC;
+            const uint8_t* pr = prep + i * C::PREC;
+            const float4* A = reinterpret_cast<const float4*>(pr + C::PR_A);  // alpha k, e, k, alpha
+            const float2* B = reinterpret_cast<const float2*>(pr + C::PR_B);  // q, b
             const size_t t = (size_t)ts + i;
             cp_async_wait_all();
             float SP[RJ][kMC];
-            get_slice<DK>(SP, spb + (i & 1) * C::S4, warp, lane);
-            if (i > 0) copy_slice_async<DK>(spb + ((i - 1) & 1) * C::S4, sprev(i - 1), warp, lane);
-            else if (s > 0) copy_slice_async<DK>(spb + C::S4, ckpt(s - 1), warp, lane);
-            cp_async_commit();
-
-            const auto rv = row_vals<DK, DV, T>(rec, lane);
-            float dO[16];
-            ld16(reinterpret_cast<const float*>(rec + C::OFF_DO) + kMC * warp, dO);
+            get_slice<DK>(SP, spb, warp, lane);
+            float dO[kMC];
+            ldc(reinterpret_cast<const float*>(pr + C::PR_DO) + kMC * warp, dO);
             // dS += q dO^T; column sums r = S'^T k, dx = dS^T k, dr = -dS^T e
-            float a[3][16];
+            float a[3][kMC];
 #pragma unroll
-            for (int mm = 0; mm < 16; ++mm) {
-                float ar = 0.f, ax = 0.f, ad = 0.f;
+            for (int mm = 0; mm < kMC; ++mm) a[0][mm] = a[1][mm] = a[2][mm] = 0.f;
 #pragma unroll
-                for (int j = 0; j < RJ; ++j) {
-                    const float d = fmaf(rv.q[j], dO[mm], dS[j][mm]);
+            for (int j = 0; j < RJ; ++j) {
+                const float4 rw = A[lane + 32 * j];
+                const float qj = B[lane + 32 * j].x;
+#pragma unroll
+                for (int mm = 0; mm < kMC; ++mm) {
+                    const float d = fmaf(qj, dO[mm], dS[j][mm]);
                     dS[j][mm] = d;
-                    ar = fmaf(rv.al[j] * rv.k[j], SP[j][mm], ar);
-                    ax = fmaf(rv.k[j], d, ax);
-                    ad = fmaf(-rv.e[j], d, ad);
+                    a[0][mm] = fmaf(rw.x, SP[j][mm], a[0][mm]);
+                    a[1][mm] = fmaf(rw.z, d, a[1][mm]);
+                    a[2][mm] = fmaf(-rw.y, d, a[2][mm]);
                 }
-                a[0][mm] = ar; a[1][mm] = ax; a[2][mm] = ad;
             }
+            // every S_prev value has been consumed: fetch the next token's into the buffer
+            if (i > 0) copy_slice_async<DK>(spb, sprev(i - 1), warp, lane);
+            else if (s > 0) copy_slice_async<DK>(spb, ckpt(s - 1), warp, lane);
+            cp_async_commit();
             col_reduce<3>(a, lane);
             __syncwarp();
-            if (!(lane & 1)) {
-                const int mc = lane >> 1, m = kMC * warp + mc;
+            if (!(lane & 3)) {
+                const int mc = lane >> 2, m = kMC * warp + mc;
                 col[mc] = a[0][0];
                 col[kMC + mc] = a[2][0];
                 const size_t tv = t * p.h_v + h;
-                bp.dw[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(rec + C::OFF_V)[m]);
-                bp.dv[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(rec + C::OFF_W)[m]);
+                bp.dw[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_V)[m]);
+                bp.dv[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_W)[m]);
             }
             __syncwarp();
-            float r[16], dr[16], x[16];
-            ld16(col, r);
-            ld16(col + kMC, dr);
-            {
-                float v[16], w[16];
-                ld16(reinterpret_cast<const T*>(rec + C::OFF_V) + kMC * warp, v);
-                ld16(reinterpret_cast<const T*>(rec + C::OFF_W) + kMC * warp, w);
-#pragma unroll
-                for (int mm = 0; mm < 16; ++mm) x[mm] = w[mm] * v[mm];
-            }
+            float r[kMC], dr[kMC], x[kMC];
+            ldc(col, r);
+            ldc(col + kMC, dr);
+            ldc(reinterpret_cast<const float*>(pr + C::PR_X) + kMC * warp, x);
             float rdo = 0.f, xdo = 0.f;
 #pragma unroll
-            for (int mm = 0; mm < 16; ++mm) {
+            for (int mm = 0; mm < kMC; ++mm) {
                 rdo = fmaf(r[mm], dO[mm], rdo);
                 xdo = fmaf(x[mm], dO[mm], xdo);
             }
@@ -376,30 +379,32 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             float* pw = part + ((size_t)pb * C::NW + warp) * 4 * DK;
 #pragma unroll
             for (int j = 0; j < RJ; ++j) {
+                const float4 rw = A[lane + 32 * j];
+                const float bj = B[lane + 32 * j].y;
                 float pde = 0.f, pdk = 0.f, pdr = 0.f, pda = 0.f, psd = 0.f;
 #pragma unroll
-                for (int mm = 0; mm < 16; ++mm) {
+                for (int mm = 0; mm < kMC; ++mm) {
                     const float d = dS[j][mm], sp = SP[j][mm];
-                    const float dsp = fmaf(rv.k[j], dr[mm], d);
+                    const float dsp = fmaf(rw.z, dr[mm], d);
                     pde = fmaf(d, r[mm], pde);
                     pdk = fmaf(d, x[mm], pdk);
                     pdr = fmaf(sp, dr[mm], pdr);
                     pda = fmaf(dsp, sp, pda);
                     psd = fmaf(sp, dO[mm], psd);
-                    dS[j][mm] = rv.al[j] * dsp;
+                    dS[j][mm] = rw.w * dsp;
                 }
                 const int c = lane + 32 * j;
-                pw[c] = fmaf(rv.al[j], psd, fmaf(-rv.e[j], rdo, rv.k[j] * xdo));  // dq
-                pw[DK + c] = fmaf(rv.al[j], pdr, fmaf(-rv.b[j], pde, pdk));       // dk
-                pw[2 * DK + c] = -rv.k[j] * pde;                                   // db
-                pw[3 * DK + c] = rv.al[j] * pda;                                   // dlog_alpha
+                pw[c] = fmaf(rw.w, psd, fmaf(-rw.y, rdo, rw.z * xdo));  // dq
+                pw[DK + c] = fmaf(rw.w, pdr, fmaf(-bj, pde, pdk));      // dk
+                pw[2 * DK + c] = -rw.z * pde;                            // db
+                pw[3 * DK + c] = rw.w * pda;                             // dlog_alpha
             }
             __syncthreads();
-            const float* pr = part + (size_t)pb * C::NW * 4 * DK;
+            const float* pr_sum = part + (size_t)pb * C::NW * 4 * DK;
             for (int o = threadIdx.x; o < 4 * DK; o += C::NT) {
                 float sum = 0.f;
 #pragma unroll
-                for (int w = 0; w < C::NW; ++w) sum += pr[w * 4 * DK + o];
+                for (int w = 0; w < C::NW; ++w) sum += pr_sum[w * 4 * DK + o];
                 const int which = o / DK, c = o - which * DK;
                 const size_t iq = (t * p.h_qk + g) * DK + c, iv = (t * p.h_v + h) * DK + c;
                 if (which == 0) {
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
 #pragma unroll
         for (int j = 0; j < RJ; ++j)
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
+            for (int qq = 0; qq < kQ; ++qq)
                 dst[gidx<DV>(warp, lane, j, qq)] =
                     make_float4(dS[j][4 * qq], dS[j][4 * qq + 1], dS[j][4 * qq + 2], dS[j][4 * qq + 3]);
     }

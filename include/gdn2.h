@@ -184,7 +184,7 @@ GDN2_API gdn2_status gdn2_chunk_fwd_prologue(const gdn2_shape* shape,
  *   dS0 (nullable) [n_seq, h_v, dk, dv].
  * The pages describe the forward recurrence only (they state the model was trained, which
  * needs these); the derivation is the chain rule through the per-token update, in fp32.
- * One CTA runs per (sequence, value head), each warp owning 16 value columns of the state
+ * One CTA runs per (sequence, value head), each warp owning 8 value columns of the state
  * in registers: a forward pass stores the state at every 8th token, then, from the end, each
  * 8-token sub-chunk's states are recomputed into a scratch area and its tokens walked
  * backwards.
