@@ -174,15 +174,16 @@ __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t
                                          int warp) {
     using C = Cfg<DK, DV, T>;
     const float4* A = reinterpret_cast<const float4*>(pr + C::PR_A);
+    float4 rw[C::RJ];  // alpha k, e, k, alpha of this lane's rows
+#pragma unroll
+    for (int j = 0; j < C::RJ; ++j) rw[j] = A[lane + 32 * j];
     float a[1][kMC];
 #pragma unroll
     for (int mm = 0; mm < kMC; ++mm) a[0][mm] = 0.f;
 #pragma unroll
-    for (int j = 0; j < C::RJ; ++j) {
-        const float ak = A[lane + 32 * j].x;
+    for (int j = 0; j < C::RJ; ++j)
 #pragma unroll
-        for (int mm = 0; mm < kMC; ++mm) a[0][mm] = fmaf(ak, S[j][mm], a[0][mm]);
-    }
+        for (int mm = 0; mm < kMC; ++mm) a[0][mm] = fmaf(rw[j].x, S[j][mm], a[0][mm]);
     col_reduce<1>(a, lane);
     __syncwarp();
     if (!(lane & 3)) col[lane >> 2] = a[0][0];
@@ -191,11 +192,10 @@ __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t
     ldc(col, r);
     ldc(reinterpret_cast<const float*>(pr + C::PR_X) + kMC * warp, x);
 #pragma unroll
-    for (int j = 0; j < C::RJ; ++j) {
-        const float4 rw = A[lane + 32 * j];  // alpha k, e, k, alpha
+    for (int j = 0; j < C::RJ; ++j)
 #pragma unroll
-        for (int mm = 0; mm < kMC; ++mm) S[j][mm] = fmaf(rw.z, x[mm], fmaf(-rw.y, r[mm], rw.w * S[j][mm]));
-    }
+        for (int mm = 0; mm < kMC; ++mm)
+            S[j][mm] = fmaf(rw[j].z, x[mm], fmaf(-rw[j].y, r[mm], rw[j].w * S[j][mm]));
 }
 
 // A thread's slice of a state in its own order: float4 index of (row group j, column quad qq).

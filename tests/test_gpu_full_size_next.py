@@ -1,0 +1,134 @@
+"""Full-size parity of the backward, the fused pre-processing and the serving decode.
+
+Each path runs on the GPU (through the C ABI) over the whole workload in the launch
+configuration the benchmark times; the oracle recomputes sampled (sequence, head) pairs one
+by one and the sampled outputs are compared element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_160_b200 import workloads as W
+from tests.parity import TOL, rel_err
+
+pytestmark = pytest.mark.gpu
+
+PREFILL = "prefill_b8_h16_t4096"
+DECODE = "decode_256seq_h32"
+
+
+@pytest.fixture(scope="module")
+def g():
+    import gated_delta_rule_160_b200 as g
+    g.load_library()
+    assert torch.cuda.is_available()
+    return g
+
+
+def _slice(d, n, h, T):
+    """Tokens of sequence n (all sequences T long) and value head h = query/key head h."""
+    s = slice(n * T, (n + 1) * T)
+    return {key: d[key][s, h:h + 1].cpu() for key in ("q", "k", "v", "log_alpha", "b", "w")}
+
+
+def _S0(d, n, h):
+    return None if d["S0"] is None else d["S0"][n:n + 1, h:h + 1].cpu()
+
+
+def test_backward_full_size_sampled(g):
+    """gdn2_chunk_bwd on all 8 x 16 x 4096 token-heads; the oracle differentiates (sequence,
+    head) pairs (0, 0) and (7, 15) one at a time (query/key head = value head here)."""
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, "cuda")
+    dO = torch.randn(d["v"].shape, generator=torch.Generator(device="cuda").manual_seed(wl.seed + 29),
+                     device="cuda")
+    got = g.gdn2_chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], dO, S0=d["S0"],
+                           n_seq=d["n_seq"])
+    torch.cuda.synchronize()
+    names = ["dq", "dk", "dv", "dlog_alpha", "db", "dw"]
+    cols = {name: ([], []) for name in names + ["dS0"]}
+    T = wl.T
+    for n, h in [(0, 0), (7, 15)]:
+        x = _slice(d, n, h, T)
+        ref = oracle.bwd_ref(x["q"], x["k"], x["v"], x["log_alpha"], x["b"], x["w"],
+                             dO[n * T:(n + 1) * T, h:h + 1].cpu(), S0=_S0(d, n, h), n_seq=1)
+        for name, a, r in zip(names, got[:6], ref[:6]):
+            cols[name][0].append(a[n * T:(n + 1) * T, h])
+            cols[name][1].append(r[:, 0])
+        cols["dS0"][0].append(got[6][n, h])
+        cols["dS0"][1].append(ref[6][0, 0])
+    for name, (a, r) in cols.items():
+        err = rel_err(torch.stack(a), np.stack(r))
+        print(f"backward full size: {name} err {err:.3e}")
+        assert err <= 1e-4, name  # fp32 arithmetic
+
+
+def test_prologue_full_size_sampled(g):
+    """gdn2_chunk_fwd_prologue on the 8 x 16 x 4096 workload from raw bf16 projections (the
+    recipe of the benchmark's fused pre-processing leg); oracle: prologue_ref then fwd_ref on
+    (sequence, head) pairs (0, 0) and (7, 15)."""
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, "cuda")
+    T_all = int(sum(d["lengths"]))
+    gen = torch.Generator(device="cuda").manual_seed(wl.seed + 17)
+    rn = lambda *shp: torch.randn(*shp, generator=gen, device="cuda").to(wl.dtype)
+    raw = dict(q=rn(T_all, wl.h_qk, wl.dk), k=rn(T_all, wl.h_qk, wl.dk), a=rn(T_all, wl.h_v, wl.dk),
+               b=rn(T_all, wl.h_v, wl.dk), w=rn(T_all, wl.h_v, wl.dv))
+    o, st = g.gdn2_chunk_fwd(raw["q"], raw["k"], d["v"], raw["a"], raw["b"], raw["w"], S0=d["S0"],
+                             n_seq=d["n_seq"], prologue=True)
+    torch.cuda.synchronize()
+    T = wl.T
+    f32 = lambda x: np.asarray(x, dtype=np.float32)
+    o_got, o_ref, s_got, s_ref = [], [], [], []
+    for n, h in [(0, 0), (7, 15)]:
+        s = slice(n * T, (n + 1) * T)
+        q, k, la, b, w = oracle.prologue_ref(raw["q"][s, h:h + 1], raw["k"][s, h:h + 1], raw["a"][s, h:h + 1],
+                                             raw["b"][s, h:h + 1], raw["w"][s, h:h + 1])
+        ro, rs = oracle.fwd_ref(f32(q), f32(k), d["v"][s, h:h + 1].float().cpu().numpy(), f32(la), f32(b), f32(w),
+                                S0=_S0(d, n, h), n_seq=1, bf16=False)
+        o_got.append(o[s, h])
+        o_ref.append(ro[:, 0])
+        s_got.append(st[n, h])
+        s_ref.append(rs[0, 0])
+    eo = rel_err(torch.stack(o_got), np.stack(o_ref))
+    es = rel_err(torch.stack(s_got), np.stack(s_ref))
+    tol = TOL[torch.bfloat16]
+    print(f"prologue full size: o err {eo:.3e}, S_T err {es:.3e} (tol {tol})")
+    assert eo <= tol and es <= tol
+
+
+def test_serving_decode_full_size_sampled(g):
+    """gdn2_decode_multi on all 256 x 32 states at seeded-random slots of a 512-state pool,
+    4 tokens per sequence and step (the benchmark's serving leg), three steps; the oracle
+    replays sampled (sequence, head) pairs as 12-token sequences from the slot's state."""
+    wl = W.WORKLOADS[DECODE]
+    N, n_tok, steps = wl.n_seq, 4, 3
+    pool = torch.zeros((2 * N, wl.h_v, wl.dk, wl.dv), dtype=torch.float32, device="cuda")
+    perm = torch.randperm(2 * N, generator=torch.Generator().manual_seed(wl.seed))[:N]
+    S_init = W.decode_state(wl, "cuda")
+    pool[perm.to("cuda")] = S_init
+    slots = perm.to(torch.int32).to("cuda")
+    ins, outs = [], []
+    for s_ in range(steps):
+        t_ = W.token_inputs(N * n_tok, wl.h_qk, wl.h_v, wl.dk, wl.dv, wl.dtype, "cuda", wl.seed * 7919 + s_)
+        x = {key: t.view(N, n_tok, *t.shape[1:]) for key, t in t_.items()}
+        o, _ = g.gdn2_decode_multi(*(x[key] for key in ("q", "k", "v", "log_alpha", "b", "w")), pool, slots=slots)
+        ins.append(x)
+        outs.append(o)
+    torch.cuda.synchronize()
+    tol = TOL[torch.float32]  # fp32 arithmetic in the decode kernel
+    o_got, o_ref, s_got, s_ref = [], [], [], []
+    for n, h in [(0, 0), (255, 31), (100, 17)]:
+        seq = {key: torch.cat([x[key][n, :, h:h + 1] for x in ins]).cpu()
+               for key in ("q", "k", "v", "log_alpha", "b", "w")}
+        ro, rs = oracle.fwd_ref(seq["q"], seq["k"], seq["v"], seq["log_alpha"], seq["b"], seq["w"],
+                                S0=S_init[n:n + 1, h:h + 1].cpu(), n_seq=1)
+        o_got.append(torch.cat([o[n, :, h] for o in outs]))
+        o_ref.append(ro[:, 0])
+        s_got.append(pool[int(perm[n]), h])
+        s_ref.append(rs[0, 0])
+    eo = rel_err(torch.stack(o_got), np.stack(o_ref))
+    es = rel_err(torch.stack(s_got), np.stack(s_ref))
+    print(f"serving decode full size: o err {eo:.3e}, S err {es:.3e} (tol {tol})")
+    assert eo <= tol and es <= tol
