@@ -49,13 +49,6 @@ struct BwdParams {
     int atomic_qk;           // dq, dk accumulate (groups of value heads)
 };
 
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 // kMC consecutive fp32 values (16-byte aligned); a warp reading one address broadcasts.
 __device__ __forceinline__ void ldc(const float* p, float (&o)[kMC]) {
 #pragma unroll
@@ -177,13 +170,16 @@ __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t
     float4 rw[C::RJ];  // alpha k, e, k, alpha of this lane's rows
 #pragma unroll
     for (int j = 0; j < C::RJ; ++j) rw[j] = A[lane + 32 * j];
+    // column pairs (mm, mm + 1) in packed two-wide arithmetic
     float a[1][kMC];
 #pragma unroll
-    for (int mm = 0; mm < kMC; ++mm) a[0][mm] = 0.f;
+    for (int pp = 0; pp < kMC / 2; ++pp) {
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < C::RJ; ++j)
-#pragma unroll
-        for (int mm = 0; mm < kMC; ++mm) a[0][mm] = fmaf(rw[j].x, S[j][mm], a[0][mm]);
+        for (int j = 0; j < C::RJ; ++j) acc = ffma2(dup2(rw[j].x), make_float2(S[j][2 * pp], S[j][2 * pp + 1]), acc);
+        a[0][2 * pp] = acc.x;
+        a[0][2 * pp + 1] = acc.y;
+    }
     col_reduce<1>(a, lane);
     __syncwarp();
     if (!(lane & 3)) col[lane >> 2] = a[0][0];
@@ -194,8 +190,13 @@ __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t
 #pragma unroll
     for (int j = 0; j < C::RJ; ++j)
 #pragma unroll
-        for (int mm = 0; mm < kMC; ++mm)
-            S[j][mm] = fmaf(rw[j].z, x[mm], fmaf(-rw[j].y, r[mm], rw[j].w * S[j][mm]));
+        for (int pp = 0; pp < kMC / 2; ++pp) {
+            const float2 sj = fmul2(dup2(rw[j].w), make_float2(S[j][2 * pp], S[j][2 * pp + 1]));
+            const float2 sn = ffma2(dup2(rw[j].z), make_float2(x[2 * pp], x[2 * pp + 1]),
+                                    ffma2(dup2(-rw[j].y), make_float2(r[2 * pp], r[2 * pp + 1]), sj));
+            S[j][2 * pp] = sn.x;
+            S[j][2 * pp + 1] = sn.y;
+        }
 }
 
 // A thread's slice of a state in its own order: float4 index of (row group j, column quad qq).
@@ -335,20 +336,32 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             ldc(reinterpret_cast<const float*>(pr + C::PR_DO) + kMC * warp, dO);
             // dS += q dO^T; column sums r = S'^T k, dx = dS^T k, dr = -dS^T e
             float a[3][kMC];
+            {
+                float2 acc[3][kMC / 2];
 #pragma unroll
-            for (int mm = 0; mm < kMC; ++mm) a[0][mm] = a[1][mm] = a[2][mm] = 0.f;
+                for (int pp = 0; pp < kMC / 2; ++pp) acc[0][pp] = acc[1][pp] = acc[2][pp] = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int j = 0; j < RJ; ++j) {
-                const float4 rw = A[lane + 32 * j];
-                const float qj = B[lane + 32 * j].x;
+                for (int j = 0; j < RJ; ++j) {
+                    const float4 rw = A[lane + 32 * j];
+                    const float2 qj = dup2(B[lane + 32 * j].x), ak = dup2(rw.x), kk = dup2(rw.z), ne = dup2(-rw.y);
 #pragma unroll
-                for (int mm = 0; mm < kMC; ++mm) {
-                    const float d = fmaf(qj, dO[mm], dS[j][mm]);
-                    dS[j][mm] = d;
-                    a[0][mm] = fmaf(rw.x, SP[j][mm], a[0][mm]);
-                    a[1][mm] = fmaf(rw.z, d, a[1][mm]);
-                    a[2][mm] = fmaf(-rw.y, d, a[2][mm]);
+                    for (int pp = 0; pp < kMC / 2; ++pp) {
+                        const float2 d = ffma2(qj, make_float2(dO[2 * pp], dO[2 * pp + 1]),
+                                               make_float2(dS[j][2 * pp], dS[j][2 * pp + 1]));
+                        dS[j][2 * pp] = d.x;
+                        dS[j][2 * pp + 1] = d.y;
+                        acc[0][pp] = ffma2(ak, make_float2(SP[j][2 * pp], SP[j][2 * pp + 1]), acc[0][pp]);
+                        acc[1][pp] = ffma2(kk, d, acc[1][pp]);
+                        acc[2][pp] = ffma2(ne, d, acc[2][pp]);
+                    }
                 }
+#pragma unroll
+                for (int v = 0; v < 3; ++v)
+#pragma unroll
+                    for (int pp = 0; pp < kMC / 2; ++pp) {
+                        a[v][2 * pp] = acc[v][pp].x;
+                        a[v][2 * pp + 1] = acc[v][pp].y;
+                    }
             }
             // every S_prev value has been consumed: fetch the next token's into the buffer
             if (i > 0) copy_slice_async<DK>(spb, sprev(i - 1), warp, lane);
@@ -381,18 +394,25 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             for (int j = 0; j < RJ; ++j) {
                 const float4 rw = A[lane + 32 * j];
                 const float bj = B[lane + 32 * j].y;
-                float pde = 0.f, pdk = 0.f, pdr = 0.f, pda = 0.f, psd = 0.f;
+                const float2 kk = dup2(rw.z), al = dup2(rw.w);
+                float2 pde2 = make_float2(0.f, 0.f), pdk2 = pde2, pdr2 = pde2, pda2 = pde2, psd2 = pde2;
 #pragma unroll
-                for (int mm = 0; mm < kMC; ++mm) {
-                    const float d = dS[j][mm], sp = SP[j][mm];
-                    const float dsp = fmaf(rw.z, dr[mm], d);
-                    pde = fmaf(d, r[mm], pde);
-                    pdk = fmaf(d, x[mm], pdk);
-                    pdr = fmaf(sp, dr[mm], pdr);
-                    pda = fmaf(dsp, sp, pda);
-                    psd = fmaf(sp, dO[mm], psd);
-                    dS[j][mm] = rw.w * dsp;
+                for (int pp = 0; pp < kMC / 2; ++pp) {
+                    const float2 d = make_float2(dS[j][2 * pp], dS[j][2 * pp + 1]);
+                    const float2 sp = make_float2(SP[j][2 * pp], SP[j][2 * pp + 1]);
+                    const float2 dr2 = make_float2(dr[2 * pp], dr[2 * pp + 1]);
+                    const float2 dsp = ffma2(kk, dr2, d);
+                    pde2 = ffma2(d, make_float2(r[2 * pp], r[2 * pp + 1]), pde2);
+                    pdk2 = ffma2(d, make_float2(x[2 * pp], x[2 * pp + 1]), pdk2);
+                    pdr2 = ffma2(sp, dr2, pdr2);
+                    pda2 = ffma2(dsp, sp, pda2);
+                    psd2 = ffma2(sp, make_float2(dO[2 * pp], dO[2 * pp + 1]), psd2);
+                    const float2 nd = fmul2(al, dsp);
+                    dS[j][2 * pp] = nd.x;
+                    dS[j][2 * pp + 1] = nd.y;
                 }
+                const float pde = pde2.x + pde2.y, pdk = pdk2.x + pdk2.y, pdr = pdr2.x + pdr2.y;
+                const float pda = pda2.x + pda2.y, psd = psd2.x + psd2.y;
                 const int c = lane + 32 * j;
                 pw[c] = fmaf(rw.w, psd, fmaf(-rw.y, rdo, rw.z * xdo));  // dq
                 pw[DK + c] = fmaf(rw.w, pdr, fmaf(-bj, pde, pdk));      // dk

@@ -4,13 +4,16 @@
     python -m gated_delta_rule_160_b200.profile_case --kernel decode --n-seq 64 --iters 3
     python -m gated_delta_rule_160_b200.profile_case --kernel bwd --n-seq 2 --T 1024 --iters 2
     python -m gated_delta_rule_160_b200.profile_case --kernel grouped --n-seq 2 --T 8192 --iters 3
+    python -m gated_delta_rule_160_b200.profile_case --kernel serving --n-seq 64 --iters 3
 
 ``chunk`` runs gdn2_chunk_fwd on the first ``n-seq`` sequences of the 16-head, T=4096,
 d=128 bf16 prefill workload (2 sequences: 268 MB of inputs, larger than L2; ``T`` cuts them); ``decode``
 runs gdn2_decode_step on ``n-seq`` sequences of the 32-head decode workload; ``bwd`` runs
 gdn2_chunk_bwd (gradients of sum(o * dO)) on the prefill workload's first ``n-seq``
 sequences; ``grouped`` runs gdn2_chunk_fwd on the grouped-head workload (16 query/key heads
-shared by 32 value heads, with an initial state), its sequences cut to ``T`` tokens. Each
+shared by 32 value heads, with an initial state), its sequences cut to ``T`` tokens;
+``serving`` runs gdn2_decode_multi (4 tokens per sequence) on ``n-seq`` sequences of the
+32-head decode workload whose states sit at seeded-random slots of a pool twice as large. Each
 kernel is launched ``iters`` times; profile the last launches (ncu -s / -c).
 """
 import argparse
@@ -23,7 +26,7 @@ from gated_delta_rule_160_b200 import workloads as W
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--kernel", choices=["chunk", "decode", "bwd", "grouped"], default="chunk")
+    ap.add_argument("--kernel", choices=["chunk", "decode", "bwd", "grouped", "serving"], default="chunk")
     ap.add_argument("--n-seq", type=int, default=2)
     ap.add_argument("--T", type=int, default=None, help="tokens per sequence (chunk, bwd, grouped)")
     ap.add_argument("--iters", type=int, default=3)
@@ -51,6 +54,18 @@ def main():
         for _ in range(a.iters):
             G.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=d["S0"], n_seq=a.n_seq,
                              o=o, S_T=S_T)
+    elif a.kernel == "serving":
+        wl = W.WORKLOADS["decode_256seq_h32"]
+        N, n_tok = a.n_seq, 4
+        pool = torch.zeros((2 * N, wl.h_v, wl.dk, wl.dv), dtype=torch.float32, device="cuda")
+        perm = torch.randperm(2 * N, generator=torch.Generator().manual_seed(wl.seed))[:N]
+        pool[perm.to("cuda")] = W.decode_state(wl, "cuda", n_seq=N)
+        slots = perm.to(torch.int32).to("cuda")
+        t_ = W.token_inputs(N * n_tok, wl.h_qk, wl.h_v, wl.dk, wl.dv, wl.dtype, "cuda", wl.seed * 7919)
+        x = {k: t.view(N, n_tok, *t.shape[1:]) for k, t in t_.items()}
+        o = torch.empty((N, n_tok, wl.h_v, wl.dv), dtype=torch.float32, device="cuda")
+        for _ in range(a.iters):
+            G.gdn2_decode_multi(*(x[k] for k in ("q", "k", "v", "log_alpha", "b", "w")), pool, slots=slots, o=o)
     else:
         wl = W.WORKLOADS["decode_256seq_h32"]
         S = W.decode_state(wl, "cuda", n_seq=a.n_seq)
