@@ -390,7 +390,9 @@ def main():
                              "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flop x 1965 MHz",
                              "algorithmic_flops_per_launch": bflops,
                              "hbm": {"achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
-                                     "algorithmic_bytes_per_launch": bbytes}}}
+                                     "algorithmic_bytes_per_launch": bbytes,
+                                     "traffic": recorded_traffic("chunk_bwd_prefill_b8_h16_t4096.md",
+                                                                 "gated_delta_rule_160_b200/csrc/backward.cu")}}}
     del dO_b, ws_b
 
     # ---------------- grouped heads: 16 query/key heads shared by 32 value heads, with S0
@@ -488,7 +490,9 @@ def main():
                           "n_seq": dwl.n_seq, "heads": dwl.h_v, "n_tok": SERVING_TOKENS,
                           "pool_slots": 2 * dwl.n_seq},
                "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s", "frac": sach / hbm,
-                            "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                            "traffic": recorded_traffic("decode_multi_serving_256seq_h32.md",
+                                                        "gated_delta_rule_160_b200/csrc/decode.cu"),
+                            "peak_source": f"{peak_src} hbm_gbs",
                             "algorithmic_bytes_per_launch": sbytes}}
     del pool, srv_in, so
 
