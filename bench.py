@@ -35,6 +35,8 @@ PREFILL = "prefill_b8_h16_t4096"
 DECODE = "decode_256seq_h32"
 GROUPED = "grouped_b2_qk16_v32_t32768"
 GROUPED_TIMED_STEPS = 5
+VARLEN = "varlen_64seq_h16"
+VARLEN_TIMED_STEPS = 3
 # fp32 SIMT peak for the backward's per-token adjoint: 148 SMs x 128 fp32 lanes x 2 flop
 # (one FMA) per clock at the 1965 MHz maximum SM clock
 FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -426,6 +428,38 @@ def main():
                             "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": gbytes}}
     del gd, g_o, g_S
 
+    # ---------------- packed sequences of mixed lengths (cu_seqlens), longest first
+    vwl = W.WORKLOADS[VARLEN]
+    vd = W.prefill_inputs(vwl, dev)
+    v_o = torch.empty(vd["v"].shape, dtype=torch.float32, device=dev)
+    v_S = torch.empty((len(vd["lengths"]), vwl.h_v, vwl.dk, vwl.dv), dtype=torch.float32, device=dev)
+    sh_v = G.make_shape(vd["q"], vd["v"], len(vd["lengths"]), torch.float32)
+    ws_v = torch.empty(max(1, G.gdn2_chunk_fwd_workspace_size(sh_v, True)), dtype=torch.uint8, device=dev)
+    vstep = lambda: G.gdn2_chunk_fwd(vd["q"], vd["k"], vd["v"], vd["log_alpha"], vd["b"], vd["w"],
+                                     cu_seqlens=vd["cu_seqlens"], o=v_o, S_T=v_S, workspace=ws_v, stream=stream)
+    for _ in range(3):
+        vstep()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(VARLEN_TIMED_STEPS):
+        vstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    vms = max_over_ranks(e0.elapsed_time(e1) / VARLEN_TIMED_STEPS, world)
+    v_T = int(sum(vd["lengths"]))
+    vbytes = prefill_bytes(vwl, vd["lengths"])
+    vach = vbytes / (vms / 1000.0) / 1e9
+    varlen = {"metric": "GDN-2 chunk-fwd tokens/s, packed mixed lengths", "value": world * v_T / (vms / 1000.0),
+              "unit": "tokens/s", "ms_per_step": vms, "steps": VARLEN_TIMED_STEPS,
+              "config": {"workload": VARLEN, "sequences": len(vd["lengths"]), "tokens": v_T,
+                         "lengths": f"{min(vd['lengths'])}..{max(vd['lengths'])}", "heads": vwl.h_v,
+                         "dk": vwl.dk, "dv": vwl.dv},
+              "roofline": {"bound": "hbm", "achieved": vach, "peak": hbm, "unit": "GB/s", "frac": vach / hbm,
+                           "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
+                           "algorithmic_bytes_per_launch": vbytes}}
+    del vd, v_o, v_S, ws_v
+
     # ---------------- decode (the second metric)
     dwl = W.WORKLOADS[DECODE]
     S = W.decode_state(dwl, dev)
@@ -549,6 +583,7 @@ def main():
             "prefill_prologue": prologue,
             "backward": backward,
             "grouped": grouped,
+            "varlen": varlen,
             "e2e": e2e,
             "cpu_baseline": base,
             "clocks": clocks.summary(),
