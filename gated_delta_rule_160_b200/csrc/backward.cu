@@ -105,7 +105,8 @@ struct Cfg {
     static constexpr int SM_SP = SM_PREP + kL * PREC;             // [S4] float4: S_prev
     static constexpr int SM_PART = SM_SP + S4 * 16;               // [2][NW][4][DK] f32: row partials
     static constexpr int SM_COL = SM_PART + 2 * NW * 4 * DK * 4;  // [NW][2][kMC] f32: r, dr
-    static constexpr int SMEM = SM_COL + NW * 2 * kMC * 4;
+    static constexpr int SM_R = SM_COL + NW * 2 * kMC * 4;        // [kL][DV] f32: r of each token
+    static constexpr int SMEM = SM_R + kL * DV * 4;
 };
 
 // Queue (cp.async) the raw inputs of tokens [ts, ts + len) into a token buffer.
@@ -164,7 +165,7 @@ __device__ void prepare(const uint8_t* raw, uint8_t* prep, int len, bool with_dO
 // One forward token on this thread's slice S (key rows lane + 32 j, the warp's kMC columns).
 template <int DK, int DV, typename T>
 __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t* pr, float* col, int lane,
-                                         int warp) {
+                                         int warp, float* rkeep = nullptr) {
     using C = Cfg<DK, DV, T>;
     const float4* A = reinterpret_cast<const float4*>(pr + C::PR_A);
     float4 rw[C::RJ];  // alpha k, e, k, alpha of this lane's rows
@@ -182,7 +183,10 @@ __device__ __forceinline__ void fwd_step(float (&S)[DK / 32][kMC], const uint8_t
     }
     col_reduce<1>(a, lane);
     __syncwarp();
-    if (!(lane & 3)) col[lane >> 2] = a[0][0];
+    if (!(lane & 3)) {
+        col[lane >> 2] = a[0][0];
+        if (rkeep) rkeep[kMC * warp + (lane >> 2)] = a[0][0];  // the token's r, kept for its adjoint
+    }
     __syncwarp();
     float r[kMC], x[kMC];
     ldc(col, r);
@@ -261,6 +265,7 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
     float* part = reinterpret_cast<float*>(smem + C::SM_PART);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float* col = reinterpret_cast<float*>(smem + C::SM_COL) + warp * 2 * kMC;  // r, dr of the warp's columns
+    float* rkeep = reinterpret_cast<float*>(smem + C::SM_R);                    // [kL][DV]: r of each token
 
     const Params& p = bp.f;
     const int item = blockIdx.x;
@@ -318,10 +323,25 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
         // into the S_prev buffer for token ts + len - 1.
         get_slice<DK>(S, spb, warp, lane);
         for (int i = 0; i + 1 < len; ++i) {
-            fwd_step<DK, DV, T>(S, prep + i * C::PREC, col, lane, warp);
+            fwd_step<DK, DV, T>(S, prep + i * C::PREC, col, lane, warp, rkeep + i * DV);
             if (i + 2 < len) put_slice<DK>(scr(i), S, warp, lane);
         }
         put_slice<DK>(spb, S, warp, lane);
+        {   // r of the last token, from its S_prev (in S now)
+            const float4* A = reinterpret_cast<const float4*>(prep + (len - 1) * C::PREC + C::PR_A);
+            float a[1][kMC];
+#pragma unroll
+            for (int pp = 0; pp < kMC / 2; ++pp) {
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int j = 0; j < RJ; ++j)
+                    acc = ffma2(dup2(A[lane + 32 * j].x), make_float2(S[j][2 * pp], S[j][2 * pp + 1]), acc);
+                a[0][2 * pp] = acc.x;
+                a[0][2 * pp + 1] = acc.y;
+            }
+            col_reduce<1>(a, lane);
+            if (!(lane & 3)) rkeep[(len - 1) * DV + kMC * warp + (lane >> 2)] = a[0][0];
+        }
         // S_prev of token ts + i (i < len - 1): the checkpoint for i = 0, else scratch state i - 1
         auto sprev = [&](int i) -> const float4* { return i == 0 ? ckpt(s) : scr(i - 1); };
         for (int i = len - 1; i >= 0; --i) {
@@ -334,29 +354,32 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             get_slice<DK>(SP, spb, warp, lane);
             float dO[kMC];
             ldc(reinterpret_cast<const float*>(pr + C::PR_DO) + kMC * warp, dO);
-            // dS += q dO^T; column sums r = S'^T k, dx = dS^T k, dr = -dS^T e
-            float a[3][kMC];
-            {
-                float2 acc[3][kMC / 2];
+            // dS += q dO^T; column sums dx = dS^T k, dr = -dS^T e
+            // (r = S'^T k of this token was kept by the recompute)
+            float a[2][kMC];
+            float4 rws[RJ];  // alpha k, e, k, alpha of this lane's rows, for both loops
 #pragma unroll
-                for (int pp = 0; pp < kMC / 2; ++pp) acc[0][pp] = acc[1][pp] = acc[2][pp] = make_float2(0.f, 0.f);
+            for (int j = 0; j < RJ; ++j) rws[j] = A[lane + 32 * j];
+            {
+                float2 acc[2][kMC / 2];
+#pragma unroll
+                for (int pp = 0; pp < kMC / 2; ++pp) acc[0][pp] = acc[1][pp] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < RJ; ++j) {
-                    const float4 rw = A[lane + 32 * j];
-                    const float2 qj = dup2(B[lane + 32 * j].x), ak = dup2(rw.x), kk = dup2(rw.z), ne = dup2(-rw.y);
+                    const float4 rw = rws[j];
+                    const float2 qj = dup2(B[lane + 32 * j].x), kk = dup2(rw.z), ne = dup2(-rw.y);
 #pragma unroll
                     for (int pp = 0; pp < kMC / 2; ++pp) {
                         const float2 d = ffma2(qj, make_float2(dO[2 * pp], dO[2 * pp + 1]),
                                                make_float2(dS[j][2 * pp], dS[j][2 * pp + 1]));
                         dS[j][2 * pp] = d.x;
                         dS[j][2 * pp + 1] = d.y;
-                        acc[0][pp] = ffma2(ak, make_float2(SP[j][2 * pp], SP[j][2 * pp + 1]), acc[0][pp]);
-                        acc[1][pp] = ffma2(kk, d, acc[1][pp]);
-                        acc[2][pp] = ffma2(ne, d, acc[2][pp]);
+                        acc[0][pp] = ffma2(kk, d, acc[0][pp]);
+                        acc[1][pp] = ffma2(ne, d, acc[1][pp]);
                     }
                 }
 #pragma unroll
-                for (int v = 0; v < 3; ++v)
+                for (int v = 0; v < 2; ++v)
 #pragma unroll
                     for (int pp = 0; pp < kMC / 2; ++pp) {
                         a[v][2 * pp] = acc[v][pp].x;
@@ -367,19 +390,18 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             if (i > 0) copy_slice_async<DK>(spb, sprev(i - 1), warp, lane);
             else if (s > 0) copy_slice_async<DK>(spb, ckpt(s - 1), warp, lane);
             cp_async_commit();
-            col_reduce<3>(a, lane);
+            col_reduce<2>(a, lane);
             __syncwarp();
             if (!(lane & 3)) {
                 const int mc = lane >> 2, m = kMC * warp + mc;
-                col[mc] = a[0][0];
-                col[kMC + mc] = a[2][0];
+                col[kMC + mc] = a[1][0];
                 const size_t tv = t * p.h_v + h;
-                bp.dw[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_V)[m]);
-                bp.dv[tv * DV + m] = a[1][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_W)[m]);
+                bp.dw[tv * DV + m] = a[0][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_V)[m]);
+                bp.dv[tv * DV + m] = a[0][0] * to_f32(reinterpret_cast<const T*>(tb + i * C::REC + C::OFF_W)[m]);
             }
             __syncwarp();
             float r[kMC], dr[kMC], x[kMC];
-            ldc(col, r);
+            ldc(rkeep + i * DV + kMC * warp, r);
             ldc(col + kMC, dr);
             ldc(reinterpret_cast<const float*>(pr + C::PR_X) + kMC * warp, x);
             float rdo = 0.f, xdo = 0.f;
@@ -392,7 +414,7 @@ __global__ void __launch_bounds__(Cfg<DK, DV, T>::NT, 1) chunk_bwd_kernel(const 
             float* pw = part + ((size_t)pb * C::NW + warp) * 4 * DK;
 #pragma unroll
             for (int j = 0; j < RJ; ++j) {
-                const float4 rw = A[lane + 32 * j];
+                const float4 rw = rws[j];
                 const float bj = B[lane + 32 * j].y;
                 const float2 kk = dup2(rw.z), al = dup2(rw.w);
                 float2 pde2 = make_float2(0.f, 0.f), pdk2 = pde2, pdr2 = pde2, pda2 = pde2, psd2 = pde2;
