@@ -239,6 +239,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
     if (it < n_items) issue(it);
     cp_async_commit();
     while (it < n_items) {
+        const int nx = next_active(it + gridDim.x);  // its slot lookup overlaps the wait below
         cp_async_wait_all();
         __syncthreads();  // this item's raw rows are in; the previous item's readers are done
         float4 s[RPT];
@@ -269,7 +270,6 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
             sx[idx] = wv * to_f32(reinterpret_cast<const T*>(rec + C::RV)[c]);
         }
         __syncthreads();  // the raw rows are consumed, and so is each thread's state buffer
-        const int nx = next_active(it + gridDim.x);
         if (nx < n_items) issue(nx);
         cp_async_commit();
 
