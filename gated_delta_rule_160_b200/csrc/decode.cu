@@ -274,7 +274,6 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
         cp_async_commit();
 
         const int n = it / p.h_v, h = it % p.h_v;
-        float* S = state_of(it);
         // q . (b (.) k) and q . k of every token (and |q|, |k| with the fused pre-processing):
         // warp t takes token t
         for (int t = warp; t < n_tok; t += NT / 32) {
@@ -379,6 +378,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
                 o[3] = from_f32<TO>(pq.w - qe * r.w + qk * x.w);
             }
         }
+        float* S = state_of(it);
 #pragma unroll
         for (int i = 0; i < RPT; ++i) __stcs(reinterpret_cast<float4*>(S + (size_t)(RPT * rq + i) * DV + col), s[i]);
         it = nx;
