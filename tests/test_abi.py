@@ -100,3 +100,29 @@ def test_decode_multi_rejects_before_device_work(lib):
     assert call(sh, 2, 4) == 1 and b"not n_seq * n_tok" in lib.gdn2_last_error_string()
     assert call(sh, 3, 3) == 1 and b"n_slots = 3 too small" in lib.gdn2_last_error_string()
     assert call(sh, 3, 4) == 1 and b"q is NULL" in lib.gdn2_last_error_string()
+
+
+def test_chunk_bwd_rejects_before_device_work(lib):
+    import gated_delta_rule_160_b200 as g
+
+    def call(sh, ptr=None, ws=None, ws_bytes=0):
+        p = ctypes.c_void_p(ptr) if ptr else None
+        return lib.gdn2_chunk_bwd(ctypes.byref(sh) if sh is not None else None, *([p] * 6), None, None, p, None,
+                                  *([p] * 6), None, ws, ws_bytes, None)
+
+    assert call(None) == 1 and b"shape is NULL" in lib.gdn2_last_error_string()
+    assert call(_shape(g, dk=96)) == 2 and b"dk = 96" in lib.gdn2_last_error_string()
+    assert call(_shape(g, h_qk=2, h_v=3)) == 1
+    assert call(_shape(g)) == 1 and b"q is NULL" in lib.gdn2_last_error_string()
+    assert call(_shape(g), ptr=0x1008) == 1 and b"16-byte aligned" in lib.gdn2_last_error_string()
+
+
+def test_chunk_bwd_workspace_size(lib):
+    """Checkpoints every 8 tokens (slots n + t0 / 8 + sub-chunk, at most ceil(T / 8) + N) and a
+    7-state scratch per (sequence, value head), fp32 states, rounded up to 256 bytes."""
+    import gated_delta_rule_160_b200 as g
+    assert lib.gdn2_chunk_bwd_workspace_size(None) == 0
+    sh = _shape(g, n_seq=2, T_total=100, h_qk=1, h_v=2, dk=64, dv=64)
+    state = 64 * 64 * 4
+    expect = (-(-100 // 8) + 2) * 2 * state + 2 * 2 * 7 * state
+    assert lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(sh)) == -(-expect // 256) * 256
