@@ -6,7 +6,11 @@ memory and streams only. There is no CPU fallback: if the library is missing or 
 load, importing the functions below raises.
 
     gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, ...) -> (o, S_T)
+        (prologue=True: raw projections in, the pre-processing fused)
     gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None) -> o     (S updated in place)
+    gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, ...) -> (o, S_steps)
+    gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, ...)
+        -> (dq, dk, dv, dlog_alpha, db, dw, dS0)
 """
 from __future__ import annotations
 
@@ -21,8 +25,10 @@ LIB_PATH = os.path.join(HERE, "libgdn2.so")
 GDN2_F32, GDN2_BF16 = 0, 1
 GDN2_DECODE_MAX_TOKENS = 8  # tokens per sequence in one gdn2_decode_multi call (gdn2.h)
 STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED", 3: "GDN2_ERR_CUDA"}
-ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_decode_step",
-                 "gdn2_chunk_fwd_noalloc", "gdn2_last_error_string", "gdn2_version")
+ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_chunk_fwd_prologue",
+                 "gdn2_chunk_fwd_noalloc", "gdn2_decode_step", "gdn2_decode_multi",
+                 "gdn2_decode_multi_prologue", "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd",
+                 "gdn2_last_error_string", "gdn2_version")
 
 
 class Gdn2Error(RuntimeError):
