@@ -175,3 +175,99 @@ def test_chunked_backward_strong_decay():
         r = np.asarray(r, dtype=np.float64)[:, 0]
         assert np.isfinite(a).all()
         assert np.abs(a - r).max() <= 1e-9 * max(1.0, np.abs(r).max())
+
+
+def factored_backward(q, k, v, la, b, w, S0, dO, dS_T, C):
+    """The same gradients in the factored form a tensor-core kernel evaluates: per chunk,
+    operands scaled to the chunk's midpoint frame Gref = (G_0 + G_last) / 2 (Khat = K (.)
+    exp(G - Gref), Qhat likewise, Kbar = K (.) exp(Gref - G), Ebar likewise, Sref = exp(Gref)
+    (.) S), the Gram blocks and their adjoints as plain products of those operands, and the
+    frame's own adjoint dGref = rowsum(dSref (.) Sref) - colsum(dKhat (.) Khat + dQhat (.) Qhat)
+    + colsum(dKbar (.) Kbar + dEbar (.) Ebar), shared half and half by G_0 and G_last."""
+    T, dk = k.shape
+    dv = v.shape[1]
+    X = w * v
+    S = np.zeros((dk, dv)) if S0 is None else S0.copy()
+    starts = list(range(0, T, C))
+    entry = []
+    for c0 in starts:
+        c1 = min(T, c0 + C)
+        entry.append(S)
+        S = _chunk(k[c0:c1], q[c0:c1], la[c0:c1], b[c0:c1], X[c0:c1], S)["S_next"]
+    gq, gk, gla, gb, gX = (np.zeros_like(a) for a in (q, k, la, b, X))
+    dS = np.zeros((dk, dv)) if dS_T is None else dS_T.copy()
+    for ci in reversed(range(len(starts))):
+        c0 = starts[ci]
+        c1 = min(T, c0 + C)
+        n = c1 - c0
+        K, Q, Bg, Xc, S = k[c0:c1], q[c0:c1], b[c0:c1], X[c0:c1], entry[ci]
+        G = np.cumsum(la[c0:c1], axis=0)
+        Gref = 0.5 * (G[0] + G[-1])
+        E = Bg * K
+        up, dn = np.exp(G - Gref), np.exp(Gref - G)
+        Kh, Qh, Kb, Eb = K * up, Q * up, K * dn, E * dn
+        Sref = np.exp(Gref)[:, None] * S
+        strict, incl = np.tril(np.ones((n, n)), -1), np.tril(np.ones((n, n)))
+        A, B = strict * (Kh @ Eb.T), strict * (Kh @ Kb.T)
+        P, Qm = incl * (Qh @ Kb.T), incl * (Qh @ Eb.T)
+        Tm = np.linalg.inv(np.eye(n) + A)
+        Y = Kh @ Sref + B @ Xc
+        R = Tm @ Y
+        g = np.exp(G[-1])
+        tail = np.exp(G[-1][None, :] - G)
+        Kt, Et = K * tail, E * tail
+        dOc = dO[c0:c1]
+        dSp = g[:, None] * dS
+        dg = (dS * S).sum(1)
+        dKt, dEt = Xc @ dS.T, -(R @ dS.T)
+        dXc = Kt @ dS
+        dR = -(Et @ dS)
+        dQh = dOc @ Sref.T
+        dSref = Qh.T @ dOc
+        dP = incl * (dOc @ Xc.T)
+        dXc += P.T @ dOc
+        dQm = -incl * (dOc @ R.T)
+        dR -= Qm.T @ dOc
+        dTm = dR @ Y.T
+        dY = Tm.T @ dR
+        dA = -strict * (Tm.T @ dTm @ Tm.T)
+        dKh = dY @ Sref.T
+        dSref += Kh.T @ dY
+        dB = strict * (dY @ Xc.T)
+        dXc += B.T @ dY
+        dKh += dA @ Eb + dB @ Kb
+        dEb = dA.T @ Kh + dQm.T @ Qh
+        dKb = dB.T @ Kh + dP.T @ Qh
+        dQh += dP @ Kb + dQm @ Eb
+        dK = dKh * up + dKb * dn + dKt * tail
+        dQ = dQh * up
+        dE = dEb * dn + dEt * tail
+        tt = dKt * Kt + dEt * Et
+        dG = dKh * Kh + dQh * Qh - dKb * Kb - dEb * Eb - tt
+        dG[-1] += tt.sum(0) + dg * g
+        dGref = (dSref * Sref).sum(1) - (dKh * Kh + dQh * Qh).sum(0) + (dKb * Kb + dEb * Eb).sum(0)
+        dG[0] += 0.5 * dGref
+        dG[-1] += 0.5 * dGref
+        dSp += np.exp(Gref)[:, None] * dSref
+        gb[c0:c1] = dE * K
+        gla[c0:c1] = np.cumsum(dG[::-1], axis=0)[::-1]
+        gq[c0:c1], gk[c0:c1], gX[c0:c1] = dQ, dK + dE * Bg, dXc
+        dS = dSp
+    return gq, gk, gX * w, gla, gb, gX * v, dS
+
+
+@pytest.mark.parametrize("T,C", [(1, 64), (63, 64), (130, 64), (37, 8)])
+def test_factored_backward_equals_reverse_mode(T, C):
+    rng = np.random.default_rng(500 + T + C)
+    dk, dv = 8, 6
+    q, k, v, la, b, w, S0 = _rand_inputs(rng, T, 1, 1, dk, dv, S0_scale=0.3)
+    dO = rng.standard_normal((T, 1, dv))
+    dS_T = rng.standard_normal((1, 1, dk, dv))
+    ref = oracle.bwd_ref(q, k, v, la, b, w, dO, S0=S0, dS_T=dS_T, n_seq=1)
+    f = lambda x: x[:, 0].astype(np.float64)
+    got = factored_backward(f(q), f(k), f(v), f(la), f(b), f(w), S0[0, 0].astype(np.float64), dO[:, 0],
+                            dS_T[0, 0], C)
+    for name, a, r in zip(["dq", "dk", "dv", "dlog_alpha", "db", "dw", "dS0"], got, ref):
+        r = np.asarray(r, dtype=np.float64)
+        r = r[:, 0] if name != "dS0" else r[0, 0]
+        assert np.abs(a - r).max() <= 1e-9 * max(1.0, np.abs(r).max()), name
