@@ -16,18 +16,21 @@ naive = pytest.importorskip("fla.ops.kda.naive")
 torch = pytest.importorskip("torch")
 
 
-@pytest.mark.parametrize("T,H,K,V,with_S0", [(37, 2, 8, 6, True), (64, 1, 16, 16, False), (5, 3, 4, 10, True)])
-def test_oracle_equals_library_kda_reference(oracle_mod, T, H, K, V, with_S0):
-    rng = np.random.default_rng(T * 31 + H)
+@pytest.mark.parametrize("T,H,HV,K,V,with_S0", [(37, 2, 2, 8, 6, True), (64, 1, 1, 16, 16, False),
+                                                 (5, 3, 3, 4, 10, True), (16, 2, 4, 8, 6, True)])
+def test_oracle_equals_library_kda_reference(oracle_mod, T, H, HV, K, V, with_S0):
+    """The last case has two value heads per query/key head: the library groups them the
+    way the oracle does (value head h reads query/key head h // (HV / H))."""
+    rng = np.random.default_rng(T * 31 + H + HV)
     f32 = lambda x: np.asarray(x, np.float32)
     q = rng.standard_normal((T, H, K))
     k = rng.standard_normal((T, H, K))
     q /= np.linalg.norm(q, axis=-1, keepdims=True)
     k /= np.linalg.norm(k, axis=-1, keepdims=True)
-    v = rng.standard_normal((T, H, V))
-    la = -np.log1p(np.exp(rng.standard_normal((T, H, K))))
-    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, H))))
-    S0 = 0.3 * rng.standard_normal((1, H, K, V)) if with_S0 else None
+    v = rng.standard_normal((T, HV, V))
+    la = -np.log1p(np.exp(rng.standard_normal((T, HV, K))))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, HV))))
+    S0 = 0.3 * rng.standard_normal((1, HV, K, V)) if with_S0 else None
     q, k, v, la, beta = map(f32, (q, k, v, la, beta))
     S0 = None if S0 is None else f32(S0)
     b = np.repeat(beta[:, :, None], K, axis=2)
