@@ -126,3 +126,21 @@ def test_chunk_bwd_workspace_size(lib):
     state = 64 * 64 * 4
     expect = (-(-100 // 8) + 2) * 2 * state + 2 * 2 * 7 * state
     assert lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(sh)) == -(-expect // 256) * 256
+
+
+def test_cuda_failure_is_reported_as_cuda_error(lib):
+    """On a machine without a usable GPU a call that passes the host checks fails at its
+    launch: the status is GDN2_ERR_CUDA and the message carries the CUDA runtime's reason.
+    (A zero-token prefill needs no tensors, so it reaches the launch.)"""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present: the launch would succeed")
+    import gated_delta_rule_160_b200 as g
+    sh = _shape(g, n_seq=1, T_total=0, dk=128, dv=128)
+    assert lib.gdn2_chunk_fwd(ctypes.byref(sh), *([None] * 10), None, 0, None) == 3
+    msg = lib.gdn2_last_error_string()
+    assert msg.startswith(b"chunk kernel launch: ") and len(msg) > len(b"chunk kernel launch: ")
+    # the binding raises it as Gdn2Error with the same status
+    with pytest.raises(g.Gdn2Error) as e:
+        g._check(3)
+    assert e.value.status == 3
