@@ -48,7 +48,6 @@ def test_backward_oracle_equals_library_kda_autograd(oracle_mod):
     """The oracle's gradients (oracle.bwd_ref) at uniform gates against torch's reverse mode
     through the library's KDA reference: dq, dk, dv, dlog_alpha, dS0 directly, and the
     scalar gate's gradient as the sum of the erase and write gates' (beta feeds both)."""
-    import oracle
     rng = np.random.default_rng(5)
     T, H, K, V = 20, 2, 8, 6
     f32 = lambda x: np.asarray(x, np.float32)
@@ -64,7 +63,7 @@ def test_backward_oracle_equals_library_kda_autograd(oracle_mod):
     q, k, v, la, beta, S0 = map(f32, (q, k, v, la, beta, S0))
     b = np.repeat(beta[:, :, None], K, axis=2)
     w = np.repeat(beta[:, :, None], V, axis=2)
-    ref = oracle.bwd_ref(q, k, v, la, b, w, dO, S0=S0, dS_T=dS_T, n_seq=1)
+    ref = oracle_mod.bwd_ref(q, k, v, la, b, w, dO, S0=S0, dS_T=dS_T, n_seq=1)
     t = lambda x: torch.from_numpy(np.asarray(x, np.float64))[None].requires_grad_(True)
     tq, tk, tv, tg, tb = t(q), t(k), t(v), t(la), t(beta)
     ts0 = torch.from_numpy(S0.astype(np.float64)).requires_grad_(True)
