@@ -43,7 +43,8 @@ FP32_SIMT_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 SERVING_TOKENS = 4  # tokens per sequence in one serving-decode step (a verify step)
 PROLOGUE_TIMED_STEPS = 10
 BACKWARD_TIMED_STEPS = 3
-DECODE_TIMED_STEPS = 64
+DECODE_TIMED_STEPS = 512  # the decode workload's 512 consecutive steps
+SERVING_TIMED_STEPS = 64
 
 
 def parse():
@@ -119,34 +120,50 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def recorded_traffic(profile_name: str, source_rel: str):
-    """DRAM bytes per launch recorded from an ncu capture summarised in profiles/, or None
-    when the kernel source has changed since the capture (its sha256 prefix differs)."""
+def recorded_traffic(key: str):
+    """DRAM bytes per launch of an ncu capture, recorded in profiles/traffic.json under key,
+    or None when the kernel source has changed since the capture (its sha256 prefix
+    differs) or nothing is recorded."""
     import hashlib
-    import re
     try:
-        with open(os.path.join(ROOT, "profiles", profile_name)) as f:
-            text = f.read()
-        with open(os.path.join(ROOT, source_rel), "rb") as f:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[key]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    except OSError:
+    except (OSError, KeyError, ValueError):
         return None
-    m = re.search(r"traffic_bytes_per_launch=(\S+) kernel_sha256_prefix=(\w+)", text)
-    if not m or m.group(2) != sha or m.group(1) == "null":
+    if rec.get("source_sha256_16") != sha or rec.get("dram_bytes_per_launch") is None:
         return None
-    return int(m.group(1))
+    return int(rec["dram_bytes_per_launch"])
 
 
-def prefill_bytes(wl, lengths) -> int:
-    """Algorithmic bytes of one chunk-forward: every input read once, o and S_T written once;
-    q and k are counted once per query/key head (value heads in a group share them)."""
+def prefill_bytes(wl, lengths, o_bytes=None) -> int:
+    """Algorithmic bytes of one chunk-forward: every input read once, o and S_T written once
+    (S0 read once when given); q and k are counted once per query/key head (value heads in a
+    group share them). o_bytes is the size of one output element: by default that of the
+    input dtype, which is the survey's count (2048 B per token and head for bf16 inputs,
+    d = 128); the kernel writes o in fp32 (o_bytes = 4, 2304 B)."""
     es = torch.finfo(wl.dtype).bits // 8
+    ob = es if o_bytes is None else o_bytes
     T = int(sum(lengths))
-    # q, k per query/key head; v, w, b per value head; log_alpha fp32; o written as fp32
+    # q, k per query/key head; v, w, b per value head; log_alpha fp32; o
     per_token = (wl.h_qk * 2 * wl.dk * es
-                 + wl.h_v * (2 * wl.dv * es + wl.dk * es + 4 * wl.dk + 4 * wl.dv))
+                 + wl.h_v * (2 * wl.dv * es + wl.dk * es + 4 * wl.dk + ob * wl.dv))
     state = wl.n_seq * wl.h_v * wl.dk * wl.dv * 4
     return T * per_token + state * (2 if wl.S0_std else 1)
+
+
+def hbm_roofline(nbytes: int, nbytes_f32o: int, ms: float, hbm: float, peak_src: str, traffic, **extra):
+    """The HBM roofline of one chunk-forward launch of ms milliseconds: achieved = the
+    survey's algorithmic bytes / time; the same with o counted as the fp32 it is written in
+    alongside."""
+    ach = nbytes / (ms / 1000.0) / 1e9
+    ach32 = nbytes_f32o / (ms / 1000.0) / 1e9
+    r = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "traffic": traffic,
+         "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": nbytes,
+         "fp32_o": {"achieved": ach32, "frac": ach32 / hbm, "algorithmic_bytes_per_launch": nbytes_f32o}}
+    r.update(extra)
+    return r
 
 
 def prologue_bytes(wl, lengths) -> int:
@@ -325,14 +342,9 @@ def main():
     ms = max_over_ranks(ms_local, world)
     kern_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends))
     value = world * tokens_per_step / (ms / 1000.0)
-    nbytes = prefill_bytes(wl, d["lengths"])
-    achieved = nbytes / (kern_ms / 1000.0) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm,
-                "traffic": recorded_traffic("chunk_tc_prefill_b8_h16_t4096.md",
-                                            "gated_delta_rule_160_b200/csrc/chunk_tc.cu"),
-                "peak_source": f"{peak_src} hbm_gbs", "kernel": "gdn2 chunk-forward",
-                "algorithmic_bytes_per_launch": nbytes}
+    roofline = hbm_roofline(prefill_bytes(wl, d["lengths"]), prefill_bytes(wl, d["lengths"], 4), kern_ms, hbm,
+                            peak_src, recorded_traffic("chunk_tc_prefill_b8_h16_t4096"),
+                            kernel="gdn2 chunk-forward", kernel_ms=kern_ms)
 
     o_device_run = o.cpu()  # the timed prefill's output, checked against the end-to-end path below
 
@@ -395,8 +407,7 @@ def main():
                              "algorithmic_flops_per_launch": bflops,
                              "hbm": {"achieved": bach, "peak": hbm, "unit": "GB/s", "frac": bach / hbm,
                                      "algorithmic_bytes_per_launch": bbytes,
-                                     "traffic": recorded_traffic("chunk_bwd_prefill_b8_h16_t4096.md",
-                                                                 "gated_delta_rule_160_b200/csrc/backward.cu")}}}
+                                     "traffic": recorded_traffic("chunk_bwd_prefill_b8_h16_t4096")}}}
     del dO_b, ws_b
 
     # ---------------- grouped heads: 16 query/key heads shared by 32 value heads, with S0
@@ -417,17 +428,13 @@ def main():
     torch.cuda.synchronize()
     gms = max_over_ranks(e0.elapsed_time(e1) / GROUPED_TIMED_STEPS, world)
     g_T = int(sum(gd["lengths"]))
-    gbytes = prefill_bytes(gwl, gd["lengths"])
-    gach = gbytes / (gms / 1000.0) / 1e9
     grouped = {"metric": "GDN-2 chunk-fwd tokens/s, grouped heads", "value": world * g_T / (gms / 1000.0),
                "unit": "tokens/s", "ms_per_step": gms, "steps": GROUPED_TIMED_STEPS,
                "config": {"workload": GROUPED, "global_batch": gwl.n_seq, "seq_len": gwl.T, "qk_heads": gwl.h_qk,
                           "v_heads": gwl.h_v, "dk": gwl.dk, "dv": gwl.dv,
                           "bytes": "q, k counted once per query/key head"},
-               "roofline": {"bound": "hbm", "achieved": gach, "peak": hbm, "unit": "GB/s", "frac": gach / hbm,
-                            "traffic": recorded_traffic("chunk_tc_grouped_b2_qk16_v32.md",
-                                                        "gated_delta_rule_160_b200/csrc/chunk_tc.cu"),
-                            "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": gbytes}}
+               "roofline": hbm_roofline(prefill_bytes(gwl, gd["lengths"]), prefill_bytes(gwl, gd["lengths"], 4), gms,
+                                        hbm, peak_src, recorded_traffic("chunk_tc_grouped_b2_qk16_v32"))}
     del gd, g_o, g_S
 
     # ---------------- packed sequences of mixed lengths (cu_seqlens), longest first
@@ -450,24 +457,21 @@ def main():
     torch.cuda.synchronize()
     vms = max_over_ranks(e0.elapsed_time(e1) / VARLEN_TIMED_STEPS, world)
     v_T = int(sum(vd["lengths"]))
-    vbytes = prefill_bytes(vwl, vd["lengths"])
-    vach = vbytes / (vms / 1000.0) / 1e9
     varlen = {"metric": "GDN-2 chunk-fwd tokens/s, packed mixed lengths", "value": world * v_T / (vms / 1000.0),
               "unit": "tokens/s", "ms_per_step": vms, "steps": VARLEN_TIMED_STEPS,
               "config": {"workload": VARLEN, "sequences": len(vd["lengths"]), "tokens": v_T,
                          "lengths": f"{min(vd['lengths'])}..{max(vd['lengths'])}", "heads": vwl.h_v,
                          "dk": vwl.dk, "dv": vwl.dv},
-              "roofline": {"bound": "hbm", "achieved": vach, "peak": hbm, "unit": "GB/s", "frac": vach / hbm,
-                           "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
-                           "algorithmic_bytes_per_launch": vbytes}}
+              "roofline": hbm_roofline(prefill_bytes(vwl, vd["lengths"]), prefill_bytes(vwl, vd["lengths"], 4), vms,
+                                       hbm, peak_src, None)}
     del vd, v_o, v_S, ws_v
 
     # ---------------- decode (the second metric)
     dwl = W.WORKLOADS[DECODE]
     S = W.decode_state(dwl, dev)
-    dec_in = [W.decode_inputs(dwl, s, dev) for s in range(4)]
+    dec_in = [W.decode_inputs(dwl, s, dev) for s in range(8)]
     do = torch.empty(dec_in[0]["v"].shape, dtype=torch.float32, device=dev)
-    dstep = lambda i: G.gdn2_decode_step(*(dec_in[i % 4][k] for k in ("q", "k", "v", "log_alpha", "b", "w")),
+    dstep = lambda i: G.gdn2_decode_step(*(dec_in[i % 8][k] for k in ("q", "k", "v", "log_alpha", "b", "w")),
                                          S, o=do, stream=stream)
     for i in range(5):
         dstep(i)
@@ -487,8 +491,7 @@ def main():
                          "dv": dwl.dv, "state_bytes": dwl.n_seq * dwl.h_v * dwl.dk * dwl.dv * 4},
               "roofline": {"bound": "hbm", "achieved": dach, "peak": hbm, "unit": "GB/s",
                            "frac": dach / hbm,
-                           "traffic": recorded_traffic("decode_256seq_h32.md",
-                                                       "gated_delta_rule_160_b200/csrc/decode.cu"),
+                           "traffic": recorded_traffic("decode_256seq_h32"),
                            "peak_source": f"{peak_src} hbm_gbs",
                            "algorithmic_bytes_per_launch": dbytes}}
     del S, dec_in
@@ -511,23 +514,22 @@ def main():
     torch.cuda.synchronize()
     barrier(world)
     e0.record(stream)
-    for i in range(DECODE_TIMED_STEPS):
+    for i in range(SERVING_TIMED_STEPS):
         sstep(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    sms = max_over_ranks(e0.elapsed_time(e1) / DECODE_TIMED_STEPS, world)
+    sms = max_over_ranks(e0.elapsed_time(e1) / SERVING_TIMED_STEPS, world)
     sbytes = serving_bytes(dwl, SERVING_TOKENS)
     sach = sbytes / (sms / 1000.0) / 1e9
     serving = {"metric": "GDN-2 serving decode tokens/s",
                "value": world * dwl.n_seq * SERVING_TOKENS / (sms / 1000.0), "unit": "tokens/s",
-               "ms_per_step": sms, "steps": DECODE_TIMED_STEPS,
+               "ms_per_step": sms, "steps": SERVING_TIMED_STEPS,
                "config": {"workload": f"{DECODE}, states at seeded-random slots of a {2 * dwl.n_seq}-state "
                                       f"pool, {SERVING_TOKENS} tokens per sequence and step",
                           "n_seq": dwl.n_seq, "heads": dwl.h_v, "n_tok": SERVING_TOKENS,
                           "pool_slots": 2 * dwl.n_seq},
                "roofline": {"bound": "hbm", "achieved": sach, "peak": hbm, "unit": "GB/s", "frac": sach / hbm,
-                            "traffic": recorded_traffic("decode_multi_serving_256seq_h32.md",
-                                                        "gated_delta_rule_160_b200/csrc/decode.cu"),
+                            "traffic": recorded_traffic("decode_multi_serving_256seq_h32"),
                             "peak_source": f"{peak_src} hbm_gbs",
                             "algorithmic_bytes_per_launch": sbytes}}
     del pool, srv_in, so
@@ -590,6 +592,8 @@ def main():
         base = cpu_baseline()
 
     if rank == 0:
+        # the two headline metrics come first and last: the driver keeps the standard keys
+        # and the last 1500 characters of the line, so decode sits at its end
         line = {
             "metric": "GDN-2 chunk-fwd tokens/s", "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
@@ -600,14 +604,14 @@ def main():
                        "inputs": "bf16 q,k,v,b,w; fp32 log_alpha, state and output",
                        "l2": "inputs (1.07 GB per rank) larger than L2; no flush"},
             "roofline": roofline,
-            "decode": decode,
-            "serving_decode": serving,
-            "prefill_prologue": prologue,
-            "backward": backward,
+            "e2e": e2e,
             "grouped": grouped,
             "varlen": varlen,
-            "e2e": e2e,
+            "prefill_prologue": prologue,
+            "backward": backward,
+            "serving_decode": serving,
             "cpu_baseline": base,
+            "decode": decode,
             "clocks": clocks.summary(),
             "gpu_launches": args.steps,
         }

@@ -11,6 +11,7 @@ load, importing the functions below raises.
     gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, ...) -> (o, S_steps)
     gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, ...)
         -> (dq, dk, dv, dlog_alpha, db, dw, dS0)
+    gdn2_device_status(stream=None) -> int   (device-side error bits, read and cleared)
 """
 from __future__ import annotations
 
@@ -28,7 +29,10 @@ STATUS = {0: "GDN2_OK", 1: "GDN2_ERR_INVALID_ARG", 2: "GDN2_ERR_UNSUPPORTED", 3:
 ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_chunk_fwd_prologue",
                  "gdn2_chunk_fwd_noalloc", "gdn2_decode_step", "gdn2_decode_multi",
                  "gdn2_decode_multi_prologue", "gdn2_chunk_bwd_workspace_size", "gdn2_chunk_bwd",
-                 "gdn2_last_error_string", "gdn2_version")
+                 "gdn2_device_status", "gdn2_testing_set_wait_limit", "gdn2_last_error_string",
+                 "gdn2_version")
+# bits of the device status word (gdn2_device_status)
+GDN2_DEVICE_WAIT_TIMEOUT, GDN2_DEVICE_BAD_SEQLENS, GDN2_DEVICE_BAD_ORDER = 0x1, 0x2, 0x4
 
 
 class Gdn2Error(RuntimeError):
@@ -74,6 +78,10 @@ def load_library(path: str = LIB_PATH):
     lib.gdn2_chunk_bwd_workspace_size.argtypes = [ctypes.POINTER(Shape)]
     lib.gdn2_chunk_bwd.restype = ctypes.c_int
     lib.gdn2_chunk_bwd.argtypes = [ctypes.POINTER(Shape)] + [vp] * 17 + [vp, sz, vp]
+    lib.gdn2_device_status.restype = ctypes.c_int
+    lib.gdn2_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), vp]
+    lib.gdn2_testing_set_wait_limit.restype = None
+    lib.gdn2_testing_set_wait_limit.argtypes = [ctypes.c_ulonglong, ctypes.c_int]
     lib.gdn2_last_error_string.restype = ctypes.c_char_p
     lib.gdn2_last_error_string.argtypes = []
     lib.gdn2_version.restype = ctypes.c_int
@@ -228,3 +236,11 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=
                               _ptr(dla), _ptr(db), _ptr(dw), _ptr(dS0), _ptr(workspace),
                               ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
     return dq, dk, dv, dla, db, dw, dS0
+
+
+def gdn2_device_status(stream=None) -> int:
+    """Wait for the work queued on ``stream`` (default: the current stream) and return, then
+    clear, the device status bits set since the last call (GDN2_DEVICE_* above; 0 = none)."""
+    flags = ctypes.c_uint(0)
+    _check(load_library().gdn2_device_status(ctypes.byref(flags), _stream_handle(stream)))
+    return int(flags.value)

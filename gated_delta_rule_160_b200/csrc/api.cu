@@ -5,12 +5,19 @@
 #include <stdarg.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "internal.cuh"
 
 namespace gdn2 {
 namespace {
 
 thread_local char g_err[512] = "";
+
+// Testing hook (gdn2_testing_set_wait_limit): limit of the prefill's bounded waits, and
+// whether its producer withholds the first loads.
+std::atomic<unsigned long long> g_wait_ns{kDefaultWaitNs};
+std::atomic<int> g_withhold{0};
 
 gdn2_status fail(gdn2_status st, const char* fmt, ...) {
     va_list ap;
@@ -90,6 +97,8 @@ Params make_params(const gdn2_shape* sh, const void* q, const void* k, const voi
     p.q = q; p.k = k; p.v = v; p.log_alpha = la; p.b = b; p.w = w;
     p.S0 = S0; p.cu_seqlens = cu; p.o = o; p.S_T = S_T; p.order = nullptr;
     p.n_tok = 1; p.slots = nullptr; p.n_slots = sh->n_seq; p.S_steps = nullptr;
+    p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
+    p.test_withhold_loads = g_withhold.load(std::memory_order_relaxed);
     return p;
 }
 
@@ -105,7 +114,26 @@ extern "C" {
 
 const char* gdn2_last_error_string(void) { return g_err; }
 
-int gdn2_version(void) { return 100; }
+int gdn2_version(void) { return 200; }
+
+gdn2_status gdn2_device_status(unsigned int* flags, gdn2_stream_t stream) {
+    if (!flags) return fail(GDN2_ERR_INVALID_ARG, "flags is NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned int w[3] = {0u, 0u, 0u};
+    cudaError_t e = cudaStreamSynchronize(s);  // the work queued so far has run
+    if (e == cudaSuccess) e = read_clear_status_chunk_tc(&w[0], s);
+    if (e == cudaSuccess) e = read_clear_status_recurrent(&w[1], s);
+    if (e == cudaSuccess) e = read_clear_status_schedule(&w[2], s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the reads have landed in w
+    if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
+    *flags = w[0] | w[1] | w[2];
+    return ok();
+}
+
+void gdn2_testing_set_wait_limit(unsigned long long wait_ns, int withhold_first_load) {
+    g_wait_ns.store(wait_ns ? wait_ns : kDefaultWaitNs, std::memory_order_relaxed);
+    g_withhold.store(withhold_first_load ? 1 : 0, std::memory_order_relaxed);
+}
 
 size_t gdn2_chunk_fwd_workspace_size(const gdn2_shape* shape, int varlen) {
     if (!shape || !varlen || shape->n_seq < 1) return 0;
@@ -293,6 +321,10 @@ gdn2_status gdn2_chunk_bwd(const gdn2_shape* shape, const void* q, const void* k
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(GDN2_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
     Params p = make_params(shape, q, k, v, log_alpha, b, w, S0, cu_seqlens, nullptr, nullptr);
+    if (cu_seqlens) {
+        cudaError_t ec = launch_check_seqlens(p, reinterpret_cast<cudaStream_t>(stream));
+        if (ec != cudaSuccess) return fail(GDN2_ERR_CUDA, "cu_seqlens check kernel: %s", cudaGetErrorString(ec));
+    }
     cudaError_t e = launch_bwd(p, shape->dtype, dO, dS_T, dq, dk, dv, dlog_alpha, db, dw, dS0, workspace,
                                reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "backward kernel launch: %s", cudaGetErrorString(e));

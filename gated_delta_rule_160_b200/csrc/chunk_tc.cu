@@ -64,7 +64,6 @@ constexpr int NS = 512;           // SIMT threads (warps 0..15): prep, epilogues
 constexpr int kIssuer = NS / 32;       // warp 16 issues every MMA
 constexpr int kProducer = kIssuer + 1;  // warp 17 issues every TMA load of raw chunk rows
 constexpr int NT = NS + 64;             // threads per CTA
-constexpr uint64_t kWaitNs = 4000000000ull;  // a wait on our own MMAs that exceeds this is a fault
 constexpr float kLog2e = 1.4426950408889634f;  // cumulative log-decays are kept in base 2
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
@@ -148,7 +147,9 @@ struct RawMaps {
     CUtensorMap o;  // fp32 output, used for full chunks (box {128, 1, 32}, no swizzle)
 };
 
-__device__ unsigned int g_tc_fault = 0;
+// Device status word of this file's kernels (kStatus* bits), read and cleared by
+// gdn2_device_status.
+__device__ unsigned int g_status_tc = 0;
 
 __device__ __forceinline__ uint32_t off_rowmajor(int r, int c) {  // prep tiles, 128 channels
     return (uint32_t)((r >> 3) * 2048 + (c >> 3) * 128 + (r & 7) * 16 + (c & 7) * 2);
@@ -221,6 +222,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     const int item = blockIdx.x;
     const int n = p.order ? p.order[item / p.h_v] : item / p.h_v;
     const int h = item % p.h_v;
+    if ((unsigned)n >= (unsigned)p.n_seq) {  // a stale order entry: skip the item, touch nothing
+        if (tid == 0) atomicOr(&g_status_tc, kStatusBadOrder);
+        return;
+    }
+    const uint64_t kWaitNs = p.wait_ns;
     const int g = h / (p.h_v / p.h_qk);
     int t0, t1;
     seq_bounds(p, n, t0, t1);
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         // One thread of the producer warp stages every chunk's raw rows: q, k, b as soon as
         // the Sref MMAs of the previous chunk have read the tiles they land on, log_alpha,
         // v, w once the previous chunk's X^T P^T MMAs and its UT solve are done with theirs.
-        if (lane == 0) {
+        if (lane == 0 && !p.test_withhold_loads) {
             issue_raw_a(t0);
             issue_raw_b(t0);
             for (int ci = 0; ci + 1 < nchunks; ++ci) {
@@ -937,7 +943,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             p.S_T[soff + (size_t)c * D + L] = u[e] * exp2f(scal[256 + buf * 128 + c] - scal[buf * 128 + c]);
         }
     }
-    if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_tc_fault, 1u);
+    if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_status_tc, kStatusWaitTimeout);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1009,11 +1015,11 @@ cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s) {
     return odt == GDN2_F32 ? launch_tc_t<float, false>(p, s) : launch_tc_t<__nv_bfloat16, false>(p, s);
 }
 
-cudaError_t read_tc_fault(unsigned int* out) {
-    cudaError_t e = cudaMemcpyFromSymbol(out, g_tc_fault, sizeof(unsigned int));
+cudaError_t read_clear_status_chunk_tc(unsigned int* out, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_status_tc, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return e;
-    const unsigned int zero = 0;
-    return cudaMemcpyToSymbol(g_tc_fault, &zero, sizeof(unsigned int));
+    static const unsigned int zero = 0;
+    return cudaMemcpyToSymbolAsync(g_status_tc, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s);
 }
 
 }  // namespace gdn2

@@ -34,7 +34,19 @@ struct Params {
     // -softplus(a_raw), b, w <- sigmoid
     int prologue;
     const void* a_raw;
+    // bounded waits (tensor-core prefill): a wait longer than wait_ns is a fault; the CTA
+    // records it in the device status word, releases its tensor memory and returns
+    unsigned long long wait_ns;
+    // testing only: the prefill's producer never issues the first chunk's loads, so every
+    // wait of the CTA runs out (nothing asynchronous is in flight when it gives up)
+    int test_withhold_loads;
 };
+
+// Device status word bits (see gdn2_device_status in gdn2.h).
+constexpr unsigned int kStatusWaitTimeout = GDN2_DEVICE_WAIT_TIMEOUT;
+constexpr unsigned int kStatusBadSeqlens = GDN2_DEVICE_BAD_SEQLENS;
+constexpr unsigned int kStatusBadOrder = GDN2_DEVICE_BAD_ORDER;
+constexpr unsigned long long kDefaultWaitNs = 4000000000ull;
 
 // Pieces of the fused pre-processing, in fp32, on the special-function unit. Their errors
 // are absolute ~1e-7 (softplus: summed into log-decays) and relative ~1e-6 (sigmoid), far
@@ -112,7 +124,13 @@ cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaSt
 cudaError_t launch_varlen_order(const Params& p, int32_t* order, cudaStream_t s);
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt);
 cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);  // honours p.prologue
-cudaError_t read_tc_fault(unsigned int* out);
+// Each translation unit that can flag a device-side error keeps its own status word; these
+// queue, on stream s, a read of the word into *out (host) followed by clearing it.
+cudaError_t read_clear_status_chunk_tc(unsigned int* out, cudaStream_t s);
+cudaError_t read_clear_status_recurrent(unsigned int* out, cudaStream_t s);
+cudaError_t read_clear_status_schedule(unsigned int* out, cudaStream_t s);
+// Validate cu_seqlens on the device (flags kStatusBadSeqlens); used where no order kernel runs.
+cudaError_t launch_check_seqlens(const Params& p, cudaStream_t s);
 // Backward (gradients of the recurrence).
 size_t bwd_workspace_bytes(const gdn2_shape* sh);
 cudaError_t launch_bwd(const Params& p, gdn2_dtype dt, const float* dO, const float* dS_T, float* dq, float* dk,

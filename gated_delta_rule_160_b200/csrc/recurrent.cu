@@ -33,6 +33,10 @@ struct RecSmem {
     float red[2][2][kSplit][kCols];  // [token parity][r | p][warp][column]
 };
 
+// Device status word of this file's kernel (kStatus* bits), read and cleared by
+// gdn2_device_status.
+__device__ unsigned int g_status_rec = 0;
+
 template <int DK, typename T, typename TO>
 __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
     __shared__ RecSmem<DK> sm;
@@ -42,6 +46,10 @@ __global__ void __launch_bounds__(kCols * kSplit) recurrent_kernel(Params p) {
     const int slice = blockIdx.x;
     const int h = blockIdx.y;
     const int n = p.order ? p.order[blockIdx.z] : (int)blockIdx.z;
+    if ((unsigned)n >= (unsigned)p.n_seq) {  // a stale order entry: skip the item, touch nothing
+        if (threadIdx.x == 0) atomicOr(&g_status_rec, kStatusBadOrder);
+        return;
+    }
     const int g = h / (p.h_v / p.h_qk);
     const int col = slice * kCols + lane;
     const int row0 = warp * RPT;
@@ -150,6 +158,13 @@ cudaError_t launch_rec_dk(const Params& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t read_clear_status_recurrent(unsigned int* out, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_status_rec, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    static const unsigned int zero = 0;
+    return cudaMemcpyToSymbolAsync(g_status_rec, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s);
+}
 
 cudaError_t launch_recurrent(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s) {
     if (dt == GDN2_F32)

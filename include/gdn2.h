@@ -216,7 +216,10 @@ GDN2_API gdn2_status gdn2_chunk_bwd(const gdn2_shape* shape,
  * by every GPU that loads the library until the process exits.
  * Limits: with cu_seqlens, at most 16384 sequences per call (more: GDN2_ERR_INVALID_ARG,
  * nothing queued). All calls on a device share that array; each call writes every entry
- * it reads, but calls whose work overlaps on the GPU (concurrent streams) race on it. The
+ * it reads, but calls whose work overlaps on the GPU (concurrent streams) race on it: such
+ * an overlap can give wrong or missing results (a work item that meets an out-of-range
+ * sequence index is skipped and flags GDN2_DEVICE_BAD_ORDER), but never writes outside
+ * the caller's buffers. The
  * first call on each device looks the array up with that device current: make it before
  * any stream capture. Nothing is allocated by this call.
  */
@@ -225,6 +228,43 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
                                     const float* log_alpha, const void* b, const void* w,
                                     const float* S0, const int32_t* cu_seqlens,
                                     void* o, float* S_T, gdn2_stream_t stream);
+
+/*
+ * Device-side status. The pages describe no interface, so this is an interface choice: some
+ * errors can only be seen once the kernels run, after the call that queued them has
+ * returned GDN2_OK. The kernels record them in a status word per device (bits below), and
+ * gdn2_device_status waits for the work queued so far on `stream`, returns the bits set
+ * since the previous gdn2_device_status on this device in *flags, and clears them. It
+ * synchronises `stream` (0 = the legacy default stream); work queued on other streams is
+ * covered once it has completed.
+ *   GDN2_DEVICE_WAIT_TIMEOUT  a bounded wait inside the tensor-core prefill ran out (4 s):
+ *                             that CTA released its tensor memory and returned without
+ *                             writing its rows of o and its S_T, so the outputs of that
+ *                             call are incomplete.
+ *   GDN2_DEVICE_BAD_SEQLENS   cu_seqlens was not 0 = c_0 <= c_1 <= ... <= c_n = T_total.
+ *                             Kernels clamp every sequence to [0, T_total], so nothing is
+ *                             accessed out of bounds, but the results follow the clamped
+ *                             ranges, not the caller's intent.
+ *   GDN2_DEVICE_BAD_ORDER     a work item met a sequence index outside [0, n_seq) in the
+ *                             packed-batch order (only possible when gdn2_chunk_fwd_noalloc
+ *                             calls overlap on the GPU): that item was skipped, its outputs
+ *                             are missing, and nothing was written out of bounds.
+ * Returns GDN2_ERR_CUDA if the stream or the copies fail.
+ */
+#define GDN2_DEVICE_WAIT_TIMEOUT 0x1u
+#define GDN2_DEVICE_BAD_SEQLENS 0x2u
+#define GDN2_DEVICE_BAD_ORDER 0x4u
+GDN2_API gdn2_status gdn2_device_status(unsigned int* flags, gdn2_stream_t stream);
+
+/*
+ * Testing only: the limit of the tensor-core prefill's bounded waits for later calls from
+ * any thread (wait_ns = 0 restores the default of 4 s), and, when withhold_first_load is
+ * non-zero, a prefill whose producer never issues its first loads. With a short limit the
+ * waits then run out, the kernel records GDN2_DEVICE_WAIT_TIMEOUT and returns, which lets a
+ * test check that path without any fault: nothing asynchronous is in flight when the waits
+ * give up. Not for production use.
+ */
+GDN2_API void gdn2_testing_set_wait_limit(unsigned long long wait_ns, int withhold_first_load);
 
 /* Description of the calling thread's last failure ("" if none). Never NULL. */
 GDN2_API const char* gdn2_last_error_string(void);

@@ -144,3 +144,8 @@ def test_cuda_failure_is_reported_as_cuda_error(lib):
     with pytest.raises(g.Gdn2Error) as e:
         g._check(3)
     assert e.value.status == 3
+
+
+def test_device_status_rejects_null_flags(lib):
+    assert lib.gdn2_device_status(None, None) == 1
+    assert b"flags is NULL" in lib.gdn2_last_error_string()

@@ -97,3 +97,43 @@ def test_multi_token_equals_prefill(g):
     torch.cuda.synchronize()
     torch.testing.assert_close(o_dec.reshape(N * n_tok, H, D), o_pre, rtol=1e-4, atol=1e-5)
     torch.testing.assert_close(pool, S_pre, rtol=1e-4, atol=1e-5)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+@pytest.mark.parametrize("n_tok", [1, 4, 8])
+@pytest.mark.parametrize("want_steps", [False, True])
+def test_narrow_heads_match_oracle(g, oracle_mod, dk, dv, n_tok, want_steps):
+    """Every key/value width of the serving-decode kernels (64 and 128), 1, 4 and 8 tokens,
+    with and without the per-token states, over a pool with inactive and out-of-range slots;
+    element by element against the oracle run from each active slot's state."""
+    N, H, n_slots = 6, 2, 9
+    slots = [4, -1, 8, 0, 9, 2]  # -1 and 9 (>= n_slots) are skipped
+    d = W.token_inputs(N * n_tok, H, H, dk, dv, torch.bfloat16, "cuda", seed=50 + dk + dv + n_tok)
+    d = {k_: t.view(N, n_tok, *t.shape[1:]) for k_, t in d.items()}
+    pool = W.state_input(n_slots, H, dk, dv, 0.05, "cuda", seed=51 + n_tok)
+    before = pool.clone()
+    o = torch.full((N, n_tok, H, dv), 123.0, device="cuda")
+    slots_t = torch.tensor(slots, dtype=torch.int32, device="cuda")
+    o, steps = g.gdn2_decode_multi(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], pool,
+                                   slots=slots_t, o=o, want_steps=want_steps)
+    torch.cuda.synchronize()
+    tol = TOL[torch.float32]
+    o_got, o_ref, s_got, s_ref = [], [], [], []
+    for n, s in enumerate(slots):
+        if not 0 <= s < n_slots:
+            assert torch.all(o[n] == 123.0), "a skipped sequence's rows of o were written"
+            continue
+        ref_o, ref_s = _oracle(oracle_mod, d, n, n_tok, before[s])
+        o_got.append(o[n])
+        o_ref.append(ref_o)
+        s_got.append(pool[s])
+        s_ref.append(ref_s)
+        if want_steps:
+            for t in range(n_tok):
+                _, st = _oracle(oracle_mod, d, n, t + 1, before[s])
+                assert rel_err(steps[n, t], st) <= tol, (n, t)
+    eo = rel_err(torch.stack(o_got), np.stack(o_ref))
+    es = rel_err(torch.stack(s_got), np.stack(s_ref))
+    assert eo <= tol and es <= tol, (eo, es)
+    untouched = [s for s in range(n_slots) if s not in slots]
+    assert torch.equal(pool[untouched], before[untouched])
