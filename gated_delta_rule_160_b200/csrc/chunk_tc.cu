@@ -30,23 +30,24 @@
 // scheduler hide their latency where two did not. A seventeenth warp only issues the MMA
 // groups, each as soon as the SIMT warps signal that its operands are written, so no SIMT
 // warp waits behind the tensor pipe; an eighteenth issues the TMA loads of the next chunk's
-// raw rows as soon as their space is free. The MMAs of phases 4 and 6 run while the UT
-// solve's SIMT work proceeds:
-//   1 prep    read the chunk's raw rows (staged by TMA), cumsum log-decays, write the tiles
-//   2 Gram    3 MMAs (one full, two cross terms restricted to lanes 0..63); the X tiles are
-//             written while they run
-//   3 Gram epilogue (B, A, Qm) + fp32 blocked triangular solve for T (16 -> 32 -> 64);
-//     the P block (after its cross terms) beside the solve's first level, then MMA
-//     O^T += X^T P^T (hi / lo)
-//   4 MMA     Y^T = X^T B^T
-//   5 state epilogue: U <- f (.) U, Sref^T (bf16 hi / lo) into tensor memory
-//   6 MMA     Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (hi / lo), then U += X^T Kb
-//   7 Y^T (bf16, tensor memory)  8 MMA R^T = Y^T T^T  9 -R^T (bf16, tensor memory)
-//   10 MMA: O^T -= R^T Qm^T, U -= R^T Eb
+// raw rows as soon as their space is free. Work that does not need the state is placed
+// under the MMAs that do:
+//   1 prep    q, k, b rows (staged by TMA) -> Kh, Qh hi/lo, Kb hi/lo, Eb tiles; MMA Gram
+//   2 X = w (.) v tiles and the state epilogue (U <- f (.) U, Sref^T bf16 hi / lo into
+//     tensor memory), both under the Gram MMAs; MMAs Y^T = Sref^T Kh^T,
+//     O^T = Sref^T Qh^T (hi / lo), U += X^T Kb (hi / lo)
+//   3 Gram epilogue (B, A, Qm); MMA Y^T += X^T B^T
+//   4 UT solve T = (I + A)^-1 (16 -> 32 -> 64), the P block (after its cross terms) beside
+//     its first level; MMA O^T += X^T P^T
+//   5 Y^T (bf16, tensor memory); MMA R^T = Y^T T^T
+//   6 -R^T (bf16, tensor memory); MMAs O^T -= R^T Qm^T, U -= R^T Eb
+//   7 under those MMAs: the next chunk's cumulative log-decays and frame factors
+//   8 o epilogue (full fp32 chunks: staged in the X tiles, TMA-stored in the next chunk's
+//     prep; else plain stores)
 // Sref^T, Y^T and -R^T are A operands read from tensor memory; the others come from shared
 // memory.
-//   11 o epilogue (full fp32 chunks: one TMA store of a staged tile; else plain stores)
-// The next chunk's raw rows are staged by TMA while the current one is processed.
+// The next chunk's raw rows are staged by TMA (and prefetched into L2 one chunk earlier)
+// while the current one is processed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -88,10 +89,11 @@ constexpr uint32_t OFF_XL = 7 * kTile;   // X lo
 constexpr uint32_t OFF_RAW_Q = 0;            // bf16, 16 KB each
 constexpr uint32_t OFF_RAW_K = 1 * kTile;
 constexpr uint32_t OFF_RAW_B = 2 * kTile;
-// The o tile of a full chunk is staged as fp32 [32 tokens][128 channels] halves over Kb hi
-// and Kb lo (free once the U += X^T Kb MMAs are done) and written by two TMA stores.
-constexpr uint32_t OFF_OST0 = OFF_KBH;       // tokens 0..31, fp32, 16 KB
-constexpr uint32_t OFF_OST1 = OFF_KBL;       // tokens 32..63
+// The o tile of a full chunk is staged as fp32 [32 tokens][128 channels] halves over X hi
+// and X lo (free once the X^T Kb, X^T B^T and X^T P^T MMAs are done; rewritten after the
+// next chunk's Gram has been issued) and written by two TMA stores.
+constexpr uint32_t OFF_OST0 = OFF_XH;        // tokens 0..31, fp32, 16 KB
+constexpr uint32_t OFF_OST1 = OFF_XL;        // tokens 32..63
 // [64][64] bf16 tiles. MN-major B operands B[n=i][k=j] written by the Gram epilogue:
 //   (i/8)*1024 + (j/8)*128 + (j%8)*16 + (i%8)*2     (SBO = 1024, LBO = 128)
 constexpr uint32_t kSmall = CH * CH * 2;  // 8192
@@ -124,9 +126,10 @@ constexpr uint32_t TM_D1 = 128;  // [Y^T | O^T]
 constexpr uint32_t TM_R = 256;   // R^T
 constexpr uint32_t TM_U = 384;   // state, lanes m (value channel), cols c (key channel)
 constexpr uint32_t TM_S = 320;   // Sref^T hi as a bf16 A operand (packed pairs), 64 columns
-// Sref^T lo, over the B / A blocks of the Gram (read by its epilogue before the state
-// epilogue writes this; the next Gram comes after the Sref MMAs are done)
-constexpr uint32_t TM_SL = TM_G;
+// Sref^T lo, over the R^T columns: R^T of the previous chunk is dead once its U -= R^T Eb
+// MMAs are done (before the state epilogue writes this), and R^T of this chunk is written
+// after the Sref MMAs are done
+constexpr uint32_t TM_SL = TM_R;
 // Y^T and -R^T also serve as bf16 A operands from tensor memory, packed over the first 32
 // columns of their own fp32 accumulators (TM_D1, TM_R).
 
@@ -171,8 +174,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // about 16 significant bits.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     hi = pack_bf16(a, b);
-    const float ha = __uint_as_float(hi << 16), hb = __uint_as_float(hi & 0xffff0000u);
-    lo = pack_bf16(a - ha, b - hb);
+    // a - hi(a), b - hi(b) in one packed FMA; both differences are exact in fp32
+    const float2 r = ffma2(make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)),
+                           make_float2(-1.f, -1.f), make_float2(a, b));
+    lo = pack_bf16(r.x, r.y);
 }
 
 // 4 consecutive bf16 values (8 bytes) widened to fp32.
@@ -285,6 +290,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             tma_load_3d(sbase + OFF_RAW_B + x * 8192, &maps.b, 64 * x, h, ts, mbar(MB_RAWB));
         }
     };
+    auto prefetch_raw = [&](int ts) {  // every raw row of the chunk at token ts, into L2
+#pragma unroll
+        for (int x = 0; x < (kPro ? 2 : 4); ++x) tma_prefetch_3d(&maps.la, (kPro ? 64 : 32) * x, h, ts);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            tma_prefetch_3d(&maps.q, 64 * x, g, ts);
+            tma_prefetch_3d(&maps.k, 64 * x, g, ts);
+            tma_prefetch_3d(&maps.b, 64 * x, h, ts);
+            tma_prefetch_3d(&maps.v, 64 * x, h, ts);
+            tma_prefetch_3d(&maps.w, 64 * x, h, ts);
+        }
+    };
     if (warp == kProducer) {
         // One thread of the producer warp stages every chunk's raw rows: q, k, b as soon as
         // the Sref MMAs of the previous chunk have read the tiles they land on, log_alpha,
@@ -292,9 +309,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         if (lane == 0 && !p.test_withhold_loads) {
             issue_raw_a(t0);
             issue_raw_b(t0);
+            if (nchunks > 1) prefetch_raw(t0 + CH);
             for (int ci = 0; ci + 1 < nchunks; ++ci) {
                 const uint32_t par = (uint32_t)(ci & 1);
                 const int ts = t0 + (ci + 1) * CH;
+                // the chunk after the next one reaches L2 while this chunk is processed, so its
+                // loads, issued once their space frees up, do not wait for HBM
+                if (ci + 2 < nchunks) prefetch_raw(ts + CH);
                 if (!mbar_wait(mbar(MB_2A), par, kWaitNs)) { fault = true; break; }
                 issue_raw_b(ts);
                 if (!mbar_wait(mbar(MB_2P), par, kWaitNs) || !mbar_wait(mbar(RDY_RAWA), par, kWaitNs)) {
@@ -342,25 +363,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     }
                     mma_commit(mbar(MB_GX));
                 }
-                if (!mbar_wait(mbar(RDY_2B), par, kWaitNs)) { fault = true; break; }
-                tc_fence_after();
-                {  // Y^T = X^T B^T
-                    const uint32_t id64 = idesc_bf16(128, 64, true, true);
-#pragma unroll
-                    for (int ks = 0; ks < CH / 16; ++ks)
-                        mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_XH + ks * 4096, 2048, 128),
-                                 sdesc(sbase + OFF_B + ks * 256, 128, 1024), id64, ks > 0);
-                    mma_commit(mbar(MB_2B));
-                }
                 if (!mbar_wait(mbar(RDY_2A), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
-                {  // Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T (hi / lo); then U += X^T Kb (no state read)
+                {  // Y^T = Sref^T Kh^T, O^T = Sref^T Qh^T (hi / lo); then U += X^T Kb (no state read)
                     const uint32_t id64 = idesc_bf16(128, 64, false, false);
 #pragma unroll
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t a = tmem + TM_S + ks * 8, al = tmem + TM_SL + ks * 8;
                         const uint64_t qh = sdesc(sbase + OFF_QH + ks * 256, 128, 2048);
-                        mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id64, 1u);
+                        mma_bf16_ts(tmem + TM_D1, a, sdesc(sbase + OFF_KH + ks * 256, 128, 2048), id64, ks > 0);
                         mma_bf16_ts(tmem + TM_D1 + 64, a, qh, id64, ks > 0);
                         mma_bf16_ts(tmem + TM_D1 + 64, a, sdesc(sbase + OFF_QL + ks * 256, 128, 2048), id64, 1u);
                         mma_bf16_ts(tmem + TM_D1 + 64, al, qh, id64, 1u);
@@ -375,6 +386,16 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         mma_bf16(tmem + TM_U, xl, sdesc(sbase + OFF_KBH + ks * 4096, 2048, 128), id_xx, 1u);
                         mma_bf16(tmem + TM_U, xh, sdesc(sbase + OFF_KBL + ks * 4096, 2048, 128), id_xx, 1u);
                     }
+                }
+                if (!mbar_wait(mbar(RDY_2B), par, kWaitNs)) { fault = true; break; }
+                tc_fence_after();
+                {  // Y^T += X^T B^T
+                    const uint32_t id64 = idesc_bf16(128, 64, true, true);
+#pragma unroll
+                    for (int ks = 0; ks < CH / 16; ++ks)
+                        mma_bf16(tmem + TM_D1, sdesc(sbase + OFF_XH + ks * 4096, 2048, 128),
+                                 sdesc(sbase + OFF_B + ks * 256, 128, 1024), id64, 1u);
+                    mma_commit(mbar(MB_2B));
                 }
                 if (!mbar_wait(mbar(RDY_2P), par, kWaitNs)) { fault = true; break; }
                 tc_fence_after();
@@ -421,7 +442,71 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         __syncwarp();
     }
+    // Cumulative log-decays G of chunk cs, in base 2 (G log2(e)), in place over its staged
+    // log_alpha rows (tokens past the sequence end count as zero): thread (channel c, quarter
+    // cp) sums tokens 16cp .. 16cp + 15 of channel c; the totals of the earlier quarters are
+    // added where G is read. Runs for chunk 0 before the loop and for chunk c + 1 while chunk
+    // c's last MMAs run (its rows are loaded once chunk c's UT solve is done, so by then they
+    // have arrived). Returns false if its wait for the rows ran out.
+    auto scan_cumsum = [&](int cs) -> bool {
+        const int nv = min(CH, t1 - (t0 + cs * CH));
+        const bool ok = mbar_wait(mbar(MB_RAWA), (uint32_t)(cs & 1), kWaitNs);
+        const int c = L;
+        if (kPro) {
+            // bf16 pre-activations a (upper half of the area), read completely before the
+            // cumulative decay overwrites the area
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int i = 16 * cp + r;
+                x[r] = i < nv ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    smem + OFF_RAW_A + raw_off_bf16(i, c)))
+                              : 0.f;
+            }
+            bar_sync_1<NS>();
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int i = 16 * cp + r;
+                if (i < nv) acc -= softplus_log2e_f(x[r]);
+                *reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c)) = acc;
+            }
+            qtot[128 * cp + c] = acc;
+        } else {
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int i = 16 * cp + r;
+                float* gp = reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c));
+                acc = fmaf(i < nv ? *gp : 0.f, kLog2e, acc);
+                *gp = acc;
+            }
+            qtot[128 * cp + c] = acc;
+        }
+        bar_sync_1<NS>();
+        return ok;
+    };
+    // Reference frame of chunk cs (Gref, G_last) and the factors that take the state from
+    // chunk cs - 1's frame into it: exp(G_last' - Gref') (to the state itself), then
+    // exp(Gref). Two factors, not their product: with strong decay the product underflows
+    // where the scaled state does not. (S0 takes exp(Gref) alone.) After scan_cumsum(cs),
+    // while chunk cs - 1's last MMAs run; read after the next barrier.
+    auto scan_frame = [&](int cs) {
+        if (tid < D) {
+            const int c = tid, bs = cs & 1;
+            const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
+            const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
+            fscal[c] = exp2f(cs == 0 ? gref : scal[256 + (bs ^ 1) * 128 + c] - scal[(bs ^ 1) * 128 + c]);
+            fscal[128 + c] = exp2f(gref);
+            scal[bs * 128 + c] = gref;
+            scal[256 + bs * 128 + c] = glast;
+        }
+    };
     const int simt_chunks = warp < kIssuer ? nchunks : 0;
+    if (simt_chunks > 0) {
+        fault |= !scan_cumsum(0);
+        scan_frame(0);
+    }
 
     for (int ci = 0; ci < simt_chunks; ++ci) {
         const int tc0 = t0 + ci * CH;
@@ -431,65 +516,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 1. prep
         {
-            // group A: log_alpha, v, w (tokens past the sequence end count as zero); v and w
-            // are read after the Gram MMAs are under way.
-            // Cumulative log-decay G, in base 2 (G log2(e)), in place over the staged
-            // log_alpha rows: thread (channel c, quarter cp) sums tokens 16cp .. 16cp + 15 of
-            // channel c. The totals of the earlier quarters are added where G is read.
-            fault |= !mbar_wait(mbar(MB_RAWA), par, kWaitNs);
-            if (kPro) {
-                // bf16 pre-activations a (upper half of the area), read completely before
-                // the cumulative decay overwrites the area
-                const int c = L;
-                float x[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int i = 16 * cp + r;
-                    x[r] = i < nvalid ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                            smem + OFF_RAW_A + raw_off_bf16(i, c)))
-                                      : 0.f;
-                }
-                bar_sync_1<NS>();
-                float acc = 0.f;
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int i = 16 * cp + r;
-                    if (i < nvalid) acc = fmaf(-softplus_f(x[r]), kLog2e, acc);
-                    *reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c)) = acc;
-                }
-                qtot[128 * cp + c] = acc;
-            } else {
-                const int c = L;
-                float acc = 0.f;
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int i = 16 * cp + r;
-                    float* gp = reinterpret_cast<float*>(smem + OFF_RAW_LA + raw_off_f32(i, c));
-                    acc = fmaf(i < nvalid ? *gp : 0.f, kLog2e, acc);
-                    *gp = acc;
-                }
-                qtot[128 * cp + c] = acc;
-            }
-            bar_sync_1<NS>();
-            // the previous (full) chunk's o tile, staged before this barrier
-            if (kTmaStoreO<TO> && ci > 0 && tid == 0) {
-                tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tc0 - CH);
-                tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tc0 - CH / 2);
-                bulk_commit();
-            }
-            if (tid < D) {
-                const int c = tid;
-                const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
-                const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
-                // factors taking the state from the previous chunk's reference frame into
-                // this chunk's: exp(G_last' - Gref') (to the state itself), then exp(Gref).
-                // Two factors, not their product: with strong decay the product underflows
-                // where the scaled state does not. (S0 takes exp(Gref) alone.)
-                fscal[c] = exp2f(ci == 0 ? gref : scal[256 + (buf ^ 1) * 128 + c] - scal[(buf ^ 1) * 128 + c]);
-                fscal[128 + c] = exp2f(gref);
-                scal[buf * 128 + c] = gref;
-                scal[256 + buf * 128 + c] = glast;
-            }
             // group B: q, k, b; the tiles below overwrite these rows and the staged o tile
             uint2 qq[4], kq[4], bq[4];
             fault |= !mbar_wait(mbar(MB_RAWB), par, kWaitNs);
@@ -523,13 +549,18 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         *reinterpret_cast<float2*>(npart + ((ti0 + 8 * pss) * 8 + (warp & 7)) * 2) = make_float2(sq, sk);
                 }
             }
-            // the tiles below overwrite the staged o tile (over Kb hi / lo) and Eb, which the
-            // previous chunk's U -= R^T Eb MMAs read
-            if (tid == 0) bulk_wait_read0();
+            // the tiles below overwrite Eb, which the previous chunk's U -= R^T Eb MMAs read
             if (ci > 0) fault |= !mbar_wait(mbar(MB_45), par ^ 1u, kWaitNs);
             if (bar_or_1<NS>(fault)) {
                 fault = true;
                 break;
+            }
+            // the previous (full) chunk's o tile, staged in the X tiles before this barrier;
+            // its reads must be done before the X tiles are rewritten, after the Gram's issue
+            if (kTmaStoreO<TO> && ci > 0 && tid == 0) {
+                tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tc0 - CH);
+                tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tc0 - CH / 2);
+                bulk_commit();
             }
             // 1 / |q|, 1 / |k| of this thread's tokens (all 128 channels)
             float rq[4], rk[4];
@@ -544,8 +575,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                         sq += v.x + v.z;
                         sk += v.y + v.w;
                     }
-                    rq[pss] = __frcp_rn(fmaxf(sqrtf(sq), kL2NormEps));
-                    rk[pss] = __frcp_rn(fmaxf(sqrtf(sk), kL2NormEps));
+                    // 1 / max(|x|, eps) as one reciprocal square root (relative error ~2^-22)
+                    rq[pss] = rsqrtf(fmaxf(sq, kL2NormEps * kL2NormEps));
+                    rk[pss] = rsqrtf(fmaxf(sk, kL2NormEps * kL2NormEps));
                 }
             }
             // G - Gref: this thread's tokens lie in quarters 2th and 2th + 1, whose offsets
@@ -575,7 +607,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                     for (int e = 0; e < 4; ++e) {
                         qf[e] *= rq[pss];
                         kf[e] *= rk[pss];
-                        bf[e] = sigmoid_f(bf[e]);
+                        bf[e] = sigmoid_tanh_f(bf[e]);  // b only reaches the plain bf16 Eb tile
                     }
                 }
                 float kh[4], qv[4], kb[4], eb[4];
@@ -606,6 +638,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             }
         }
         fence_proxy_async_smem();
+        if (tid == 0) bulk_wait_read0();  // the staged o tile has been read out
         if (bar_or_1<NS>(fault)) { fault = true; break; }
 
         // ------------------------------------------------------------ 2. Gram MMAs
@@ -626,17 +659,64 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 for (int e = 0; e < 4; ++e) wf[e] = sigmoid_f(wf[e]);
             }
             uint2 xh, xl;
-            split2(wf[0] * vf[0], wf[1] * vf[1], xh.x, xl.x);
-            split2(wf[2] * vf[2], wf[3] * vf[3], xh.y, xl.y);
+            const float2 x01 = fmul2(make_float2(wf[0], wf[1]), make_float2(vf[0], vf[1]));
+            const float2 x23 = fmul2(make_float2(wf[2], wf[3]), make_float2(vf[2], vf[3]));
+            split2(x01.x, x01.y, xh.x, xl.x);
+            split2(x23.x, x23.y, xh.y, xl.y);
             const uint32_t o = off_rowmajor(i, c0);
             *reinterpret_cast<uint2*>(smem + OFF_XH + o) = xh;
             *reinterpret_cast<uint2*>(smem + OFF_XL + o) = xl;
         }
+        fence_proxy_async_smem();  // the X tiles are operands of the MMAs signalled below
+        // ------------------------------------------------------------ 3. state epilogue (under the Gram MMAs)
+        // Thread (lane L, quarter cp) takes key channels 32cp .. 32cp + 31.
+        {
+            const int cb = 32 * cp;
+            float u[32];
+            if (ci == 0) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = cb + e;
+                    u[e] = (p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f) * fscal[c];
+                }
+            } else {
+                tmem_ld32_wait(tmem + lane_bits + TM_U + cb, u);
+                const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
+                const float4* g4 = reinterpret_cast<const float4*>(fscal + 128 + cb);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {  // (u f) g, two columns per packed multiply
+                    const float4 f = f4[e4], gg = g4[e4];
+                    const float2 a = fmul2(fmul2(make_float2(u[4 * e4], u[4 * e4 + 1]), make_float2(f.x, f.y)),
+                                           make_float2(gg.x, gg.y));
+                    const float2 b = fmul2(fmul2(make_float2(u[4 * e4 + 2], u[4 * e4 + 3]), make_float2(f.z, f.w)),
+                                           make_float2(gg.z, gg.w));
+                    u[4 * e4] = a.x;
+                    u[4 * e4 + 1] = a.y;
+                    u[4 * e4 + 2] = b.x;
+                    u[4 * e4 + 3] = b.y;
+                }
+            }
+            tmem_st32(tmem + lane_bits + TM_U + cb, u);
+            // Sref^T as bf16 hi / lo A operands: key channels cb .. cb + 31 in columns
+            // cb/2 .. +15 of TM_S (hi) and TM_SL (lo)
+            uint32_t pk[16], pl[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) split2(u[2 * e], u[2 * e + 1], pk[e], pl[e]);
+            tmem_st16(tmem + lane_bits + TM_S + 16 * cp, pk);
+            tmem_st16(tmem + lane_bits + TM_SL + 16 * cp, pl);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        bar_sync_1<NS>();
+
+        // ------------------------------------------------------------ 4. MMAs Y^T = Sref^T Kh^T, O^T = Sref^T Qh^T, U += X^T Kb
+        if (tid == 0) mbar_arrive(mbar(RDY_2A));
+
         fault |= !mbar_wait(mbar(MB_G), par, kWaitNs);
         if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
 
-        // ------------------------------------------------------------ 3. Gram epilogue
+        // ------------------------------------------------------------ 5. Gram epilogue
         // Thread (lane L, quarter cp) takes Gram columns 32cp .. 32cp + 31: lanes 0..63 are
         // Kb rows (B, then P), lanes 64..127 Eb rows (A, then Qm); column i, row j = L % 64.
         {
@@ -673,47 +753,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         tc_fence_before();
         if (bar_or_1<NS>(fault)) { fault = true; break; }
 
-        // ------------------------------------------------------------ 4. Y^T = X^T B^T
+        // ------------------------------------------------------------ 6. MMA Y^T += X^T B^T
         if (tid == 0) mbar_arrive(mbar(RDY_2B));
-        // ------------------------------------------------------------ 5. state epilogue
-        // Thread (lane L, quarter cp) takes key channels 32cp .. 32cp + 31.
-        {
-            const int cb = 32 * cp;
-            float u[32];
-            if (ci == 0) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = cb + e;
-                    u[e] = (p.S0 ? p.S0[soff + (size_t)c * D + L] : 0.f) * fscal[c];
-                }
-            } else {
-                tmem_ld32_wait(tmem + lane_bits + TM_U + cb, u);
-                const float4* f4 = reinterpret_cast<const float4*>(fscal + cb);
-                const float4* g4 = reinterpret_cast<const float4*>(fscal + 128 + cb);
-#pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    const float4 f = f4[e4], gg = g4[e4];
-                    u[4 * e4] = u[4 * e4] * f.x * gg.x;
-                    u[4 * e4 + 1] = u[4 * e4 + 1] * f.y * gg.y;
-                    u[4 * e4 + 2] = u[4 * e4 + 2] * f.z * gg.z;
-                    u[4 * e4 + 3] = u[4 * e4 + 3] * f.w * gg.w;
-                }
-            }
-            tmem_st32(tmem + lane_bits + TM_U + cb, u);
-            // Sref^T as bf16 hi / lo A operands: key channels cb .. cb + 31 in columns
-            // cb/2 .. +15 of TM_S (hi) and TM_SL (lo)
-            uint32_t pk[16], pl[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) split2(u[2 * e], u[2 * e + 1], pk[e], pl[e]);
-            tmem_st16(tmem + lane_bits + TM_S + 16 * cp, pk);
-            tmem_st16(tmem + lane_bits + TM_SL + 16 * cp, pl);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        bar_sync_1<NS>();
-
-        // ------------------------------------------------------------ 6. Y^T += Sref^T Kh^T, O^T = Sref^T Qh^T
-        if (tid == 0) mbar_arrive(mbar(RDY_2A));
         // ------------------------------------------------------------ 3b. UT solve, while the MMAs above run
         // T = (I + A)^-1 in three levels. Level 1: the four 16 x 16 diagonal blocks by
         // column-wise forward substitution. Levels 2 and 3 join diagonal blocks of 16 into 32
@@ -802,45 +843,54 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             WT[(base + 16 + r) * WS + base + c] = -t;
         }
         bar_sync_1<NS>();
-        {   // level 3, step 1: M = A_BA T_AA (rows 32..63, cols 0..31; 2 outputs per thread)
-            const int c = tid & 31, r0 = tid >> 5;
-            float m[2] = {0.f, 0.f};
+        if (warp < 8) {
+            // level 3 on warps 0..7: T_BA = -T_BB (A_BA T_AA), lane c = column c, four rows
+            // per warp, so every value read from shared memory feeds four FMAs
+            const int c = lane, rb = 4 * warp;
+            float m[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int l4 = 0; l4 < 32; l4 += 4) {
+            for (int l4 = 0; l4 < 32; l4 += 4) {  // M = A_BA T_AA (rows rb .. rb + 3)
                 float tv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) tv[u] = WT[(l4 + u) * WS + c];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float4 a = *reinterpret_cast<const float4*>(WA + (32 + r0 + 16 * k) * WS + l4);
+                for (int k = 0; k < 4; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WA + (32 + rb + k) * WS + l4);
                     m[k] += a.x * tv[0] + a.y * tv[1] + a.z * tv[2] + a.w * tv[3];
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 2; ++k) WM[(r0 + 16 * k) * 33 + c] = m[k];
-        }
-        bar_sync_1<NS>();
-        {   // level 3, step 2: T_BA = -T_BB M (T_BB lower triangular, its upper part is zero)
-            const int c = tid & 31, r0 = tid >> 5;
-            float t[2] = {0.f, 0.f};
-#pragma unroll
-            for (int l4 = 0; l4 < 32; l4 += 4) {
+            for (int k = 0; k < 4; ++k) WM[(rb + k) * 33 + c] = m[k];
+            bar_sync_n<2, 256>();
+            // T_BA rows rb .. rb + 3 = -T_BB M; T_BB is lower triangular, so only its columns
+            // up to rb + 3 contribute
+            float t[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int l4 = 0; l4 <= rb; l4 += 4) {
                 float mv[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) mv[u] = WM[(l4 + u) * 33 + c];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const float4 a = *reinterpret_cast<const float4*>(WT + (32 + r0 + 16 * k) * WS + 32 + l4);
+                for (int k = 0; k < 4; ++k) {
+                    const float4 a = *reinterpret_cast<const float4*>(WT + (32 + rb + k) * WS + 32 + l4);
                     t[k] += a.x * mv[0] + a.y * mv[1] + a.z * mv[2] + a.w * mv[3];
                 }
             }
+            // into the bf16 T tile (K-major [i][j]): T[32 + rb + k][c]
 #pragma unroll
-            for (int k = 0; k < 2; ++k) WT[(32 + r0 + 16 * k) * WS + c] = -t[k];
-        }
-        bar_sync_1<NS>();
-        {   // T as a K-major bf16 B operand [i][j]
-            const int i = tid & 63, jg = tid >> 6;
+            for (int k = 0; k < 4; ++k) {
+                const int i = 32 + rb + k;
+                *reinterpret_cast<__nv_bfloat16*>(smem + OFF_T + (c >> 3) * 1024 + (i >> 3) * 128 + (i & 7) * 16 +
+                                                  (c & 7) * 2) = __float2bfloat16_rn(-t[k]);
+            }
+        } else {
+            // meanwhile warps 8..15 store the parts of T complete after level 2 as the K-major
+            // bf16 B operand [i][j]: rows 0..31 (all columns), rows 32..63 columns 32..63
+            const int u = tid - 256, i = u & 31, jg = u >> 5;
             store8_bf16(smem, OFF_T + jg * 1024 + (i >> 3) * 128 + (i & 7) * 16, &WT[i * WS + 8 * jg]);
+            if (u < 128) {
+                const int i2 = 32 + i, jg2 = 4 + jg;
+                store8_bf16(smem, OFF_T + jg2 * 1024 + (i2 >> 3) * 128 + (i2 & 7) * 16, &WT[i2 * WS + 8 * jg2]);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -890,6 +940,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
 
         // ------------------------------------------------------------ 10. output and state MMAs
         if (tid == 0) mbar_arrive(mbar(RDY_45));
+        if (ci + 1 < nchunks) {  // the next chunk's scan, under the O and U MMAs
+            fault |= !scan_cumsum(ci + 1);
+            scan_frame(ci + 1);
+        }
         fault |= !mbar_wait(mbar(MB_45O), par, kWaitNs);
         if (bar_or_1<NS>(fault)) { fault = true; break; }
         tc_fence_after();
@@ -900,10 +954,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             float ov[16];
             tmem_ld16_wait(tmem + lane_bits + TM_D1 + 64 + 16 * cp, ov);
             if (kTmaStoreO<TO> && nvalid == CH) {
-                // stage the fp32 tile [token][channel] in two halves over Kb hi / lo (free:
-                // the U += X^T Kb MMAs ran before the ones just waited for; Eb, which the
-                // U -= R^T Eb MMAs may still read, is untouched); TMA stores write them after
-                // the next barrier (the next chunk's scan, or the one after the loop)
+                // stage the fp32 tile [token][channel] in two halves over X hi / lo (free:
+                // every MMA that reads them ran before the ones just waited for; Eb, which
+                // the U -= R^T Eb MMAs may still read, is untouched); TMA stores write them
+                // after the next barrier (the next chunk's first, or the one after the loop)
                 float* ost = reinterpret_cast<float*>(smem + (cp < 2 ? OFF_OST0 : OFF_OST1));
 #pragma unroll
                 for (int e = 0; e < 16; ++e) ost[(16 * (cp & 1) + e) * D + L] = ov[e];

@@ -58,6 +58,24 @@ __device__ __forceinline__ float sigmoid_f(float x) {
 __device__ __forceinline__ float softplus_f(float x) {  // log(1 + e^x), without overflow
     return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
 }
+// softplus(x) log2(e) = max(x, 0) log2(e) + log2(1 + 2^(-|x| log2(e))), in base 2 throughout
+// (two special-function operations, no conversions between the bases)
+__device__ __forceinline__ float softplus_log2e_f(float x) {
+    constexpr float kL2e = 1.4426950408889634f;
+    float e, l;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-fabsf(x) * kL2e));
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.f + e));
+    return fmaf(fmaxf(x, 0.f), kL2e, l);
+}
+// sigmoid from one special-function operation: 1/2 + tanh(x / 2) / 2, with tanh.approx's
+// relative error of about 2^-11 (absolute error of the result below 2.5e-4). Used only where
+// the value is rounded to a plain bf16 operand next (2^-9), never where a hi / lo split
+// carries it.
+__device__ __forceinline__ float sigmoid_tanh_f(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
 constexpr float kL2NormEps = 1e-12f;  // q and k are divided by max(|x|_2, eps)
 
 // 16-byte asynchronous copies global -> shared (cp.async, cached in L2 only), completed per

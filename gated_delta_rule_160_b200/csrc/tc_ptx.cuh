@@ -125,6 +125,12 @@ __device__ __forceinline__ void bar_sync_1() {
     asm volatile("bar.sync 1, %0;" ::"n"(count) : "memory");
 }
 
+// Named barrier `id` (2..15) over the first `count` threads of the CTA.
+template <int id, int count>
+__device__ __forceinline__ void bar_sync_n() {
+    asm volatile("bar.sync %0, %1;" ::"n"(id), "n"(count) : "memory");
+}
+
 // Named barrier 1 over `count` threads that also returns the OR of `v` across them.
 template <int count>
 __device__ __forceinline__ bool bar_or_1(bool v) {
@@ -270,6 +276,14 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
                      reinterpret_cast<uint64_t>(tmap)),
                  "r"(x), "r"(y), "r"(z), "r"(src)
+                 : "memory");
+}
+// TMA: prefetch the box at {x, y, z} of a 3-d tensor map into L2 (no shared memory, no
+// completion to wait for; boxes outside the tensor are ignored).
+__device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(z)
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
