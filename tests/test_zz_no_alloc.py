@@ -2,8 +2,10 @@
 memory (it keeps the packed-batch scratch in a static array inside the library). Called
 through the C ABI, it must give what gdn2_chunk_fwd gives with a caller-allocated
 workspace, within the parity tolerance, on two calls in a row with different batches (the
-shared scratch keeps the previous call's contents). This file is collected last on
-purpose, and passes alone in a fresh process as well as after the other tests."""
+shared scratch keeps the previous call's contents). Nothing here depends on what ran
+before: the tests pass alone in a fresh process and after any others. The file name only
+places them last in a full run, so that a run stopping at its first failure has already
+run every other test."""
 import ctypes
 
 import numpy as np
