@@ -119,14 +119,15 @@ int gdn2_version(void) { return 200; }
 gdn2_status gdn2_device_status(unsigned int* flags, gdn2_stream_t stream) {
     if (!flags) return fail(GDN2_ERR_INVALID_ARG, "flags is NULL");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    unsigned int w[3] = {0u, 0u, 0u};
+    unsigned int w[4] = {0u, 0u, 0u, 0u};
     cudaError_t e = cudaStreamSynchronize(s);  // the work queued so far has run
     if (e == cudaSuccess) e = read_clear_status_chunk_tc(&w[0], s);
     if (e == cudaSuccess) e = read_clear_status_recurrent(&w[1], s);
     if (e == cudaSuccess) e = read_clear_status_schedule(&w[2], s);
+    if (e == cudaSuccess) e = read_clear_status_decode(&w[3], s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);  // the reads have landed in w
     if (e != cudaSuccess) return fail(GDN2_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
-    *flags = w[0] | w[1] | w[2];
+    *flags = w[0] | w[1] | w[2] | w[3];
     return ok();
 }
 
@@ -251,6 +252,9 @@ gdn2_status decode_multi(bool prologue, const gdn2_shape* shape, int n_tok, cons
                     slots ? "given" : "NULL");
     if ((long long)shape->n_seq * shape->h_v > 0x7fffffffLL || (long long)n_slots * shape->h_v > 0x7fffffffLL)
         return fail(GDN2_ERR_UNSUPPORTED, "n_seq * h_v or n_slots * h_v too large for one launch");
+    if ((long long)n_slots * shape->h_v * shape->dk > 0x7fffffffLL)  // state rows, addressed by TMA
+        return fail(GDN2_ERR_UNSUPPORTED, "n_slots * h_v * dk = %lld state rows, above 2^31 - 1",
+                    (long long)n_slots * shape->h_v * shape->dk);
     const NamedPtr ps[] = {
         {"q", q, true}, {"k", k, true}, {"v", v, true}, {prologue ? "a" : "log_alpha", la, true}, {"b", b, true},
         {"w", w, true}, {"S_pool", S_pool, true}, {"o", o, true}, {"slots", slots, false},

@@ -1060,6 +1060,8 @@ cudaError_t launch_tc_t(const Params& p, cudaStream_t s) {
 
 }  // namespace
 
+void* tensor_map_encoder() { return reinterpret_cast<void*>(encode_fn()); }
+
 bool chunk_tc_supported(const Params& p, gdn2_dtype dt) {
     return dt == GDN2_BF16 && p.dk == D && p.dv == D && p.T_total > 0;
 }

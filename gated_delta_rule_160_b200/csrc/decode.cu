@@ -15,10 +15,19 @@
 //   o  = p - (q . (b (.) k)) r + (q . k) x                  == S_new^T q
 // which reads S once; the two column sums over the key axis are combined across row
 // groups through shared memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace gdn2 {
 namespace {
+
+// Device status word of this file's kernels (kStatus* bits), read and cleared by
+// gdn2_device_status.
+__device__ unsigned int g_status_dec = 0;
+constexpr unsigned long long kDecWaitNs = 4000000000ull;  // a state load that takes longer is a fault
 
 constexpr int kThreads = 256;
 
@@ -160,15 +169,21 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(Params p) {
 
 // ---------------------------------------------------------------- several tokens per sequence
 // Thread layout: warp w owns value columns 16w .. 16w+15 over all key rows; lane l holds the
-// float4 of columns 16w + 4(l % 4) .. +3 for the RPT = dk / 8 consecutive key rows from
-// RPT (l / 4). A column sum over the key axis is then a sum within the thread and over the
-// eight lanes that share the column quad (three shuffles), so the token loop has no CTA
-// barrier. The per-row vectors (alpha, k, q, b (.) k) are staged with row RPT rq + 4j + e
-// at float index 4 (8j + rq) + e, so the eight row groups of a warp read eight consecutive
+// float4 of columns 16w + 4(l % 4) .. +3 for the RPT = dk / 8 key rows rq, rq + 8, rq + 16,
+// ... (rq = l / 4). A column sum over the key axis is then a sum within the thread and over
+// the eight lanes that share the column quad (three shuffles), so the token loop has no CTA
+// barrier. The per-row vectors (alpha, k, q, b (.) k) are staged with row 8(4j + e) + rq at
+// float index 4 (8j + rq) + e, so the eight row groups of a warp read eight consecutive
 // float4s (no bank conflicts) and a thread's RPT rows come in RPT / 4 float4 loads.
-// Shared memory, dynamic (n_tok tokens): the next item's state [RPT][threads] float4 (each
-// thread's own slots), the next item's raw token rows [n_tok][k, q, b, log_alpha or a, v, w],
-// then the current item's fp32 vectors alpha, k, q, b (.) k [n_tok][DK] and x [n_tok][DV].
+// The next item's state arrives by TMA while the current item is processed: one thread
+// issues dv / 32 box loads of [32 columns x dk rows] with the 128-byte swizzle (16-byte
+// chunk c of row r at chunk c ^ (r % 8)), so the eight rows a warp reads at once fall in
+// distinct banks. (Per-thread 16-byte copies issued 4096 copy instructions per item, and
+// their issue stalled behind the previous item's stores.)
+// Shared memory, dynamic (n_tok tokens; the base rounded up to 1024 bytes for the swizzle):
+// the next item's state [dv / 32][dk][32] fp32, swizzled; the next item's raw token rows
+// [n_tok][k, q, b, log_alpha or a, v, w]; then the current item's fp32 vectors alpha, k, q,
+// b (.) k [n_tok][DK] and x [n_tok][DV].
 template <int DK, int DV, typename T, bool kPro>
 struct MultiCfg {
     static constexpr int NT = 2 * DV, RPT = DK / 8, ES = sizeof(T);
@@ -177,19 +192,23 @@ struct MultiCfg {
     static constexpr int CK = DK * ES / 16, CA = (RV - RA) / 16, CV = DV * ES / 16;
     static constexpr int CPT = 3 * CK + CA + 2 * CV;  // 16-byte pieces per token
     static constexpr int SBUF = RPT * NT * 16;
-    static size_t smem(int n_tok) { return SBUF + (size_t)n_tok * RREC + (size_t)n_tok * (4 * DK + DV) * 4; }
+    static size_t smem(int n_tok) { return 1024 + SBUF + (size_t)n_tok * RREC + (size_t)n_tok * (4 * DK + DV) * 4; }
 };
 
 template <int DK, int DV, typename T, typename TO, bool kPro>
-__global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi_kernel(Params p) {
+__global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
+    decode_multi_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap smap) {
     using C = MultiCfg<DK, DV, T, kPro>;
     constexpr int NT = C::NT, RPT = C::RPT;
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ float dots[GDN2_DECODE_MAX_TOKENS][2];
     __shared__ float rnorm[GDN2_DECODE_MAX_TOKENS][2];
+    __shared__ __align__(8) uint64_t state_bar;  // the state's TMA loads landed
     const int n_tok = p.n_tok;
-    float4* sbuf = reinterpret_cast<float4*>(dsm);
-    uint8_t* raw = dsm + C::SBUF;
+    uint8_t* dsm_a = dsm + ((1024u - (tc::smem_u32(dsm) & 1023u)) & 1023u);
+    const uint32_t sbuf_a = tc::smem_u32(dsm_a);
+    const uint32_t bar = tc::smem_u32(&state_bar);
+    uint8_t* raw = dsm_a + C::SBUF;
     float* sa = reinterpret_cast<float*>(raw + (size_t)n_tok * C::RREC);
     float* sk = sa + n_tok * DK;
     float* sq = sk + n_tok * DK;
@@ -197,24 +216,35 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
     float* sx = se + n_tok * DK;
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int rq = lane >> 2;                          // key rows RPT rq .. RPT rq + RPT - 1
+    const int rq = lane >> 2;                          // key rows rq, rq + 8, ..., rq + 8 (RPT - 1)
     const int col = 16 * warp + 4 * (lane & 3);        // first of its four value columns
+    // this thread's float4 of row 8i + rq in the swizzled state buffer: box col / 32, chunk
+    // (col % 32) / 4 xor (row % 8) = ... xor rq
+    const uint32_t sofs = (uint32_t)(col >> 5) * (DK * 128) + (uint32_t)rq * 128 + ((((col & 31) >> 2) ^ rq) << 4);
     const int n_items = p.n_seq * p.h_v;
     auto slot_of = [&](int it) { const int nn = it / p.h_v; return p.slots ? p.slots[nn] : nn; };
-    auto next_active = [&](int it) {
+    // the next active item from it on (its slot in *slot); a negative or out-of-range slot
+    // marks an inactive sequence
+    auto next_active = [&](int it, int* slot) {
         for (; it < n_items; it += gridDim.x) {
             const int sl = slot_of(it);
-            if (sl >= 0 && sl < p.n_slots) break;  // a negative slot: an inactive sequence
+            if (sl >= 0 && sl < p.n_slots) {
+                *slot = sl;
+                break;
+            }
         }
         return it;
     };
-    auto state_of = [&](int it) { return p.S_T + ((size_t)slot_of(it) * p.h_v + it % p.h_v) * DK * DV; };
-    // queue item it's state (this thread's float4s) and raw token rows
-    auto issue = [&](int it) {
-        const float* S = state_of(it);
-#pragma unroll
-        for (int i = 0; i < RPT; ++i) cp_async16(sbuf + i * NT + tid, S + (size_t)(RPT * rq + i) * DV + col);
+    auto state_of = [&](int it, int sl) { return p.S_T + ((size_t)sl * p.h_v + it % p.h_v) * DK * DV; };
+    // queue item it's state (TMA, one thread) and raw token rows (16-byte copies)
+    auto issue = [&](int it, int sl) {
         const int nn = it / p.h_v, hh = it % p.h_v, gg = hh / (p.h_v / p.h_qk);
+        if (tid == 0) {
+            const int row0 = (sl * p.h_v + hh) * DK;
+            tc::mbar_expect_tx(bar, DK * DV * 4);
+#pragma unroll
+            for (int b = 0; b < DV / 32; ++b) tc::tma_load_2d(sbuf_a + b * DK * 128, &smap, 32 * b, row0, bar);
+        }
         for (int u = tid; u < n_tok * C::CPT; u += NT) {
             const int t = u / C::CPT, r = u - t * C::CPT;
             const size_t row = (size_t)nn * n_tok + t, rqk = row * p.h_qk + gg, rv = row * p.h_v + hh;
@@ -235,23 +265,38 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
         }
     };
 
-    int it = next_active(blockIdx.x);
-    if (it < n_items) issue(it);
+    if (tid == 0) {
+        tc::mbar_init(bar, 1);
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    int slot = 0, nslot = 0;
+    int it = next_active(blockIdx.x, &slot);
+    if (it < n_items) issue(it, slot);
     cp_async_commit();
+    uint32_t lphase = 0;  // parity of the state load being waited for
+    bool fault = false;
     while (it < n_items) {
-        const int nx = next_active(it + gridDim.x);  // its slot lookup overlaps the wait below
+        const int nx = next_active(it + gridDim.x, &nslot);  // its slot lookup overlaps the wait below
         cp_async_wait_all();
-        __syncthreads();  // this item's raw rows are in; the previous item's readers are done
+        // bounded: a load that never lands ends the kernel with a status bit, not a hang
+        if (!tc::mbar_wait(bar, lphase, kDecWaitNs)) fault = true;
+        lphase ^= 1u;
+        if (__syncthreads_or(fault)) {  // this item's rows are in; the previous item's readers are done
+            fault = true;
+            break;
+        }
         float4 s[RPT];
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) s[i] = sbuf[i * NT + tid];
+        for (int i = 0; i < RPT; ++i)
+            s[i] = *reinterpret_cast<const float4*>(dsm_a + sofs + (uint32_t)i * (8 * 128));
         for (int idx = tid; idx < n_tok * DK; idx += NT) {
             const int t = idx / DK, c = idx - t * DK;
             const uint8_t* rec = raw + t * C::RREC;
             const float kv = to_f32(reinterpret_cast<const T*>(rec + C::RK)[c]);
             const float bv = to_f32(reinterpret_cast<const T*>(rec + C::RB)[c]);
-            const int i = c % RPT;  // staged position of row c = RPT rq + 4j + e: 4 (8j + rq) + e
-            const int ps = t * DK + 4 * (8 * (i >> 2) + c / RPT) + (i & 3);
+            const int i = c >> 3;  // staged position of row c = 8 (4j + e) + rq: 4 (8j + rq) + e
+            const int ps = t * DK + 4 * (8 * (i >> 2) + (c & 7)) + (i & 3);
             sk[ps] = kv;
             sq[ps] = to_f32(reinterpret_cast<const T*>(rec + C::RQ)[c]);
             if (kPro) {
@@ -270,13 +315,15 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
             sx[idx] = wv * to_f32(reinterpret_cast<const T*>(rec + C::RV)[c]);
         }
         __syncthreads();  // the raw rows are consumed, and so is each thread's state buffer
-        if (nx < n_items) issue(nx);
+        if (nx < n_items) issue(nx, nslot);
         cp_async_commit();
 
         const int n = it / p.h_v, h = it % p.h_v;
-        // q . (b (.) k) and q . k of every token (and |q|, |k| with the fused pre-processing):
-        // warp t takes token t
-        for (int t = warp; t < n_tok; t += NT / 32) {
+        // With the fused pre-processing, |q| and |k| are needed before the token loop, so the
+        // per-token dot products q . (b (.) k), q . k and the norms are taken here (warp t takes
+        // token t); otherwise the token loop forms the dot products itself, from the rows each
+        // thread reads anyway, and this phase and its barrier are skipped.
+        for (int t = warp; kPro && t < n_tok; t += NT / 32) {
             const float *qt = sq + t * DK, *et = se + t * DK, *kt = sk + t * DK;
             float d1 = 0.f, d2 = 0.f, nq = 0.f, nk = 0.f;
             for (int c = lane; c < DK; c += 32) {
@@ -307,7 +354,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
                 dots[t][1] = d2 * s2;
             }
         }
-        __syncthreads();
+        if (kPro) __syncthreads();
         if (kPro) {  // normalise the staged q, k (and b (.) k)
             for (int idx = tid; idx < n_tok * DK; idx += NT) {
                 const int t = idx / DK;
@@ -328,11 +375,19 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
             const float4 *et = reinterpret_cast<const float4*>(se + t * DK) + rq;
             // the state as column pairs (x, y) and (z, w): packed two-wide arithmetic
             float2 r0 = make_float2(0.f, 0.f), r1 = r0, p0 = r0, p1 = r0;
+            float2 dq = make_float2(0.f, 0.f);  // this thread's rows of q . (b (.) k), q . k
 #pragma unroll
             for (int j = 0; j < RPT / 4; ++j) {
                 const float4 a4 = at[8 * j], k4 = kt[8 * j], q4 = qt[8 * j];
                 const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kvv[4] = {k4.x, k4.y, k4.z, k4.w};
                 const float qvv[4] = {q4.x, q4.y, q4.z, q4.w};
+                if (!kPro) {
+                    const float4 e4 = et[8 * j];
+                    dq = ffma2(make_float2(q4.x, q4.x), make_float2(e4.x, k4.x), dq);
+                    dq = ffma2(make_float2(q4.y, q4.y), make_float2(e4.y, k4.y), dq);
+                    dq = ffma2(make_float2(q4.z, q4.z), make_float2(e4.z, k4.z), dq);
+                    dq = ffma2(make_float2(q4.w, q4.w), make_float2(e4.w, k4.w), dq);
+                }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     float4& si = s[4 * j + e];
@@ -346,6 +401,9 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
             // sums over the eight lanes of this column quad (the other row groups)
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
+                if (!kPro)
+                    dq = fadd2(dq, make_float2(__shfl_xor_sync(0xffffffffu, dq.x, off),
+                                               __shfl_xor_sync(0xffffffffu, dq.y, off)));
                 r0 = fadd2(r0, make_float2(__shfl_xor_sync(0xffffffffu, r0.x, off), __shfl_xor_sync(0xffffffffu, r0.y, off)));
                 r1 = fadd2(r1, make_float2(__shfl_xor_sync(0xffffffffu, r1.x, off), __shfl_xor_sync(0xffffffffu, r1.y, off)));
                 p0 = fadd2(p0, make_float2(__shfl_xor_sync(0xffffffffu, p0.x, off), __shfl_xor_sync(0xffffffffu, p0.y, off)));
@@ -366,11 +424,11 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
                     const float2 s0 = ffma2(kv, x0, ffma2(ne, r0, make_float2(si.x, si.y)));
                     const float2 s1 = ffma2(kv, x1, ffma2(ne, r1, make_float2(si.z, si.w)));
                     si = make_float4(s0.x, s0.y, s1.x, s1.y);
-                    if (Ss) __stcs(reinterpret_cast<float4*>(Ss + (size_t)(RPT * rq + 4 * j + e) * DV + col), si);
+                    if (Ss) __stcs(reinterpret_cast<float4*>(Ss + (size_t)(8 * (4 * j + e) + rq) * DV + col), si);
                 }
             }
             if (rq == 0) {
-                const float qe = dots[t][0], qk = dots[t][1];
+                const float qe = kPro ? dots[t][0] : dq.x, qk = kPro ? dots[t][1] : dq.y;
                 TO* o = static_cast<TO*>(p.o) + tv * DV + col;
                 o[0] = from_f32<TO>(pq.x - qe * r.x + qk * x.x);
                 o[1] = from_f32<TO>(pq.y - qe * r.y + qk * x.y);
@@ -378,10 +436,16 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2) decode_multi
                 o[3] = from_f32<TO>(pq.w - qe * r.w + qk * x.w);
             }
         }
-        float* S = state_of(it);
+        float* S = state_of(it, slot);
 #pragma unroll
-        for (int i = 0; i < RPT; ++i) __stcs(reinterpret_cast<float4*>(S + (size_t)(RPT * rq + i) * DV + col), s[i]);
+        for (int i = 0; i < RPT; ++i) __stcs(reinterpret_cast<float4*>(S + (size_t)(8 * i + rq) * DV + col), s[i]);
         it = nx;
+        slot = nslot;
+    }
+    if (fault) {
+        if (tid == 0) atomicOr(&g_status_dec, kStatusWaitTimeout);
+        // give a load still in flight a last bounded chance to land before the CTA exits
+        if (tid == 0) tc::mbar_wait(bar, lphase ^ 1u, kDecWaitNs);
     }
 }
 
@@ -402,9 +466,22 @@ cudaError_t launch_dec_p(const Params& p, cudaStream_t st) {
     if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, C::NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // the state pool as a 2-d fp32 tensor [n_slots * h_v * dk rows][dv], in boxes of 32
+    // columns x dk rows with the 128-byte swizzle
+    const auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encoder());
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap smap;
+    cuuint64_t dims[2] = {(cuuint64_t)DV, (cuuint64_t)p.n_slots * (cuuint64_t)p.h_v * DK};
+    cuuint64_t strides[1] = {(cuuint64_t)DV * 4};
+    cuuint32_t box[2] = {32u, (cuuint32_t)DK};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (encode(&smap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.S_T, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
     const int items = p.n_seq * p.h_v;
     const int grid = items < sms * per_sm ? items : sms * per_sm;  // persistent CTAs
-    kern<<<grid, C::NT, smem, st>>>(p);
+    kern<<<grid, C::NT, smem, st>>>(p, smap);
     return cudaGetLastError();
 }
 
@@ -420,6 +497,13 @@ cudaError_t launch_dec_t(const Params& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t read_clear_status_decode(unsigned int* out, cudaStream_t s) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_status_dec, sizeof(unsigned int), 0, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    static const unsigned int zero = 0;
+    return cudaMemcpyToSymbolAsync(g_status_dec, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, s);
+}
 
 cudaError_t launch_decode(const Params& p, gdn2_dtype dt, gdn2_dtype odt, cudaStream_t s) {
     if (dt == GDN2_F32)

@@ -147,6 +147,9 @@ cudaError_t launch_chunk_tc(const Params& p, gdn2_dtype odt, cudaStream_t s);  /
 cudaError_t read_clear_status_chunk_tc(unsigned int* out, cudaStream_t s);
 cudaError_t read_clear_status_recurrent(unsigned int* out, cudaStream_t s);
 cudaError_t read_clear_status_schedule(unsigned int* out, cudaStream_t s);
+cudaError_t read_clear_status_decode(unsigned int* out, cudaStream_t s);
+// cuTensorMapEncodeTiled from the driver (as a void*; NULL if unavailable)
+void* tensor_map_encoder();
 // Validate cu_seqlens on the device (flags kStatusBadSeqlens); used where no order kernel runs.
 cudaError_t launch_check_seqlens(const Params& p, cudaStream_t s);
 // Backward (gradients of the recurrence).
