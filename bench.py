@@ -440,6 +440,19 @@ def main():
     # ---------------- packed sequences of mixed lengths (cu_seqlens), longest first
     vwl = W.WORKLOADS[VARLEN]
     vd = W.prefill_inputs(vwl, dev)
+    all_lengths = list(vd["lengths"])
+    if world > 1:
+        # one batch split across the ranks (data parallel, no exchange): each rank keeps the
+        # sequences the longest-processing-time-first shard gives it, packed anew
+        from gated_delta_rule_160_b200.sharding import pack, shard_sequences
+        mine = shard_sequences(all_lengths, world, rank)
+        ranges, cu = pack(all_lengths, mine)
+        idx = torch.cat([torch.arange(a, z, device=dev) for a, z in ranges]) if ranges else \
+            torch.zeros(0, dtype=torch.long, device=dev)
+        for k in ("q", "k", "v", "log_alpha", "b", "w"):
+            vd[k] = vd[k].index_select(0, idx).contiguous()
+        vd["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=dev)
+        vd["lengths"] = [all_lengths[i] for i in mine]
     v_o = torch.empty(vd["v"].shape, dtype=torch.float32, device=dev)
     v_S = torch.empty((len(vd["lengths"]), vwl.h_v, vwl.dk, vwl.dv), dtype=torch.float32, device=dev)
     sh_v = G.make_shape(vd["q"], vd["v"], len(vd["lengths"]), torch.float32)
@@ -456,12 +469,15 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     vms = max_over_ranks(e0.elapsed_time(e1) / VARLEN_TIMED_STEPS, world)
-    v_T = int(sum(vd["lengths"]))
-    varlen = {"metric": "GDN-2 chunk-fwd tokens/s, packed mixed lengths", "value": world * v_T / (vms / 1000.0),
+    v_T = int(sum(all_lengths))  # the whole batch, over all ranks
+    varlen = {"metric": "GDN-2 chunk-fwd tokens/s, packed mixed lengths", "value": v_T / (vms / 1000.0),
               "unit": "tokens/s", "ms_per_step": vms, "steps": VARLEN_TIMED_STEPS,
-              "config": {"workload": VARLEN, "sequences": len(vd["lengths"]), "tokens": v_T,
-                         "lengths": f"{min(vd['lengths'])}..{max(vd['lengths'])}", "heads": vwl.h_v,
-                         "dk": vwl.dk, "dv": vwl.dv},
+              "scaling": "strong" if world > 1 else "n/a",
+              "config": {"workload": VARLEN, "sequences": len(all_lengths), "tokens": v_T,
+                         "lengths": f"{min(all_lengths)}..{max(all_lengths)}", "heads": vwl.h_v,
+                         "dk": vwl.dk, "dv": vwl.dv,
+                         "parallelism": f"sequences sharded over {world} ranks (longest first)" if world > 1
+                         else "one GPU"},
               "roofline": hbm_roofline(prefill_bytes(vwl, vd["lengths"]), prefill_bytes(vwl, vd["lengths"], 4), vms,
                                        hbm, peak_src, None)}
     del vd, v_o, v_S, ws_v
