@@ -116,7 +116,9 @@ constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 10 * 128 * 4;
 constexpr uint32_t OFF_TSLOT = OFF_MBAR + 24 * 8;
-constexpr uint32_t SMEM_BYTES = OFF_TSLOT + 16;
+// fused pre-processing: 1 / max(|q|, eps) of the chunk's tokens at [0, 64), of k at [64, 128)
+constexpr uint32_t OFF_RN = OFF_TSLOT + 16;
+constexpr uint32_t SMEM_BYTES = OFF_RN + 128 * 4;
 static_assert(OFF_WM + 32 * 33 * 4 <= OFF_REG + 4 * kTile, "solve workspace overflows its region");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -502,9 +504,36 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
             scal[256 + bs * 128 + c] = glast;
         }
     };
+    // Fused pre-processing: 1 / max(|q|, eps) and 1 / max(|k|, eps) of every token of chunk
+    // cs, for its prep, into OFF_RN. Thread u of nthr (256 or 512) takes row u / (nthr / 128)
+    // (q rows of tokens 0..63, then k rows) and sums the squares of its share of the 128
+    // channels, in swizzled 16-byte pieces. Rows past the sequence end get zero (the prep
+    // zeroes those tokens anyway). Returns false if the wait for the rows ran out.
+    auto scan_norms = [&](int cs, int u, int nthr) -> bool {
+        const bool ok = mbar_wait(mbar(MB_RAWB), (uint32_t)(cs & 1), kWaitNs);
+        const int per = nthr / 128, r = u / per, s = u % per, i = r & 63, npc = 16 / per;
+        const uint8_t* row = smem + (r < 64 ? OFF_RAW_Q : OFF_RAW_K) + i * 128;
+        float ss = 0.f;
+        for (int j = 0; j < npc; ++j) {
+            const int pc = s * npc + j;  // 16-byte piece: box pc / 8, piece pc % 8 of the row
+            const uint4 v = *reinterpret_cast<const uint4*>(row + (pc >> 3) * 8192 + (((pc & 7) ^ (i & 7)) << 4));
+            float f[4], g[4];
+            unpack4_bf16(make_uint2(v.x, v.y), f);
+            unpack4_bf16(make_uint2(v.z, v.w), g);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ss = fmaf(f[e], f[e], fmaf(g[e], g[e], ss));
+        }
+        for (int off = 1; off < per; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        // 1 / max(|x|, eps) as one reciprocal square root (relative error ~2^-22)
+        if (s == 0)
+            reinterpret_cast<float*>(smem + OFF_RN)[r] =
+                i < min(CH, t1 - (t0 + cs * CH)) ? rsqrtf(fmaxf(ss, kL2NormEps * kL2NormEps)) : 0.f;
+        return ok;
+    };
     const int simt_chunks = warp < kIssuer ? nchunks : 0;
     if (simt_chunks > 0) {
-        fault |= !scan_cumsum(0);
+        if (kPro) fault |= !scan_norms(0, tid, NS);
+        fault |= !scan_cumsum(0);  // its barriers publish the norms too
         scan_frame(0);
     }
 
@@ -529,24 +558,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
                 bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
             }
+            // 1 / |q|, 1 / |k| of this thread's tokens (taken during the previous chunk's solve)
+            float rq[4], rk[4];
             if (kPro) {
-                // per-token partial sums of squares of q and k over this warp's 16 channels,
-                // into the T tile's space (idle during the prep): [token][channel group][q, k]
-                float* npart = reinterpret_cast<float*>(smem + OFF_T);
+                const float* rn = reinterpret_cast<const float*>(smem + OFF_RN);
 #pragma unroll
                 for (int pss = 0; pss < 4; ++pss) {
-                    float qf[4], kf[4];
-                    unpack4_bf16(qq[pss], qf);
-                    unpack4_bf16(kq[pss], kf);
-                    float sq = qf[0] * qf[0] + qf[1] * qf[1] + qf[2] * qf[2] + qf[3] * qf[3];
-                    float sk = kf[0] * kf[0] + kf[1] * kf[1] + kf[2] * kf[2] + kf[3] * kf[3];
-#pragma unroll
-                    for (int off = 8; off < 32; off <<= 1) {  // the four channel quads of the token
-                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
-                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
-                    }
-                    if (lane < 8)
-                        *reinterpret_cast<float2*>(npart + ((ti0 + 8 * pss) * 8 + (warp & 7)) * 2) = make_float2(sq, sk);
+                    rq[pss] = rn[ti0 + 8 * pss];
+                    rk[pss] = rn[64 + ti0 + 8 * pss];
                 }
             }
             // the tiles below overwrite Eb, which the previous chunk's U -= R^T Eb MMAs read
@@ -561,24 +580,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tc0 - CH);
                 tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tc0 - CH / 2);
                 bulk_commit();
-            }
-            // 1 / |q|, 1 / |k| of this thread's tokens (all 128 channels)
-            float rq[4], rk[4];
-            if (kPro) {
-                const float4* npart = reinterpret_cast<const float4*>(smem + OFF_T);
-#pragma unroll
-                for (int pss = 0; pss < 4; ++pss) {
-                    float sq = 0.f, sk = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {  // eight channel groups, two per float4
-                        const float4 v = npart[(ti0 + 8 * pss) * 4 + j];
-                        sq += v.x + v.z;
-                        sk += v.y + v.w;
-                    }
-                    // 1 / max(|x|, eps) as one reciprocal square root (relative error ~2^-22)
-                    rq[pss] = rsqrtf(fmaxf(sq, kL2NormEps * kL2NormEps));
-                    rk[pss] = rsqrtf(fmaxf(sk, kL2NormEps * kL2NormEps));
-                }
             }
             // G - Gref: this thread's tokens lie in quarters 2th and 2th + 1, whose offsets
             // are the totals of the quarters before them
@@ -891,6 +892,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 const int i2 = 32 + i, jg2 = 4 + jg;
                 store8_bf16(smem, OFF_T + jg2 * 1024 + (i2 >> 3) * 128 + (i2 & 7) * 16, &WT[i2 * WS + 8 * jg2]);
             }
+            // then the next chunk's q and k norms (its q, k rows have landed by now: they are
+            // loaded once this chunk's Sref MMAs are done)
+            if (kPro && ci + 1 < nchunks) fault |= !scan_norms(ci + 1, u, 256);
         }
         fence_proxy_async_smem();
         tc_fence_before();
