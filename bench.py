@@ -373,8 +373,8 @@ def main():
                 "unit": "tokens/s", "ms_per_step": pms, "steps": PROLOGUE_TIMED_STEPS,
                 "config": {"workload": f"{PREFILL} from raw projections (bf16 decay pre-activation)"},
                 "roofline": {"bound": "hbm", "achieved": pach, "peak": hbm, "unit": "GB/s", "frac": pach / hbm,
-                             "traffic": None, "peak_source": f"{peak_src} hbm_gbs",
-                             "algorithmic_bytes_per_launch": pbytes}}
+                             "traffic": recorded_traffic("chunk_tc_prologue_prefill_b8_h16_t4096"),
+                             "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": pbytes}}
     del raw
 
     # ---------------- backward (gradients of sum(o * dO)), same workload
