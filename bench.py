@@ -564,42 +564,51 @@ def main():
         # Sequence by sequence: inputs go up on `up`, the prefill runs on `stream`, o comes
         # down on `down`, so the copies of one sequence overlap the others' work (the link is
         # full duplex). Every sequence is one gdn2_chunk_fwd call on its slice of the batch.
+        # Consecutive steps overlap as a stream of batches would: a sequence's upload waits
+        # only for the previous step's prefill of that sequence (which read the device
+        # buffers it overwrites), its prefill for the previous step's download of its o.
         up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_in = [torch.cuda.Event() for _ in range(wl.n_seq)]
         ev_out = [torch.cuda.Event() for _ in range(wl.n_seq)]
+        ev_dl = [torch.cuda.Event() for _ in range(wl.n_seq)]
 
         def e2e_step():
-            up.wait_stream(stream)
             for s_ in range(wl.n_seq):
                 sl = slice(s_ * wl.T, (s_ + 1) * wl.T)
+                up.wait_event(ev_out[s_])
                 with torch.cuda.stream(up):
                     for k in names:
                         dev_in[k][sl].copy_(host[k][sl], non_blocking=True)
                     ev_in[s_].record(up)
                 stream.wait_event(ev_in[s_])
+                stream.wait_event(ev_dl[s_])
                 G.gdn2_chunk_fwd(*(dev_in[k][sl] for k in names), n_seq=1, o=o[sl], S_T=S_T[s_:s_ + 1],
                                  stream=stream)
                 ev_out[s_].record(stream)
                 down.wait_event(ev_out[s_])
                 with torch.cuda.stream(down):
                     o_host[sl].copy_(o[sl], non_blocking=True)
-            stream.wait_stream(down)
-            stream.synchronize()
+                    ev_dl[s_].record(down)
 
         for _ in range(2):
             e2e_step()
+        stream.wait_stream(down)
+        torch.cuda.synchronize()
         n_e2e = max(3, min(args.steps, 10))
         barrier(world)
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
+        up.wait_stream(stream)  # no upload of the timed steps starts before a
         for _ in range(n_e2e):
             e2e_step()
+        stream.wait_stream(down)  # b after every step's last download
         b_.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(a.elapsed_time(b_) / n_e2e, world)
         e2e = {"value": world * tokens_per_step / (ems / 1000.0), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems,
-               "steps": n_e2e, "pipeline": "per sequence: upload, prefill and download on three streams",
+               "steps": n_e2e,
+               "pipeline": "per sequence: upload, prefill and download on three streams; consecutive steps overlap",
                "o_equals_device_run": bool(torch.equal(o_host, o_device_run))}
     del o_device_run
 

@@ -27,7 +27,6 @@ namespace {
 // Device status word of this file's kernels (kStatus* bits), read and cleared by
 // gdn2_device_status.
 __device__ unsigned int g_status_dec = 0;
-constexpr unsigned long long kDecWaitNs = 4000000000ull;  // a state load that takes longer is a fault
 
 constexpr int kThreads = 256;
 
@@ -236,10 +235,11 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
         return it;
     };
     auto state_of = [&](int it, int sl) { return p.S_T + ((size_t)sl * p.h_v + it % p.h_v) * DK * DV; };
-    // queue item it's state (TMA, one thread) and raw token rows (16-byte copies)
-    auto issue = [&](int it, int sl) {
+    // queue item it's state (TMA, one thread; not when `withhold`, the testing hook) and raw
+    // token rows (16-byte copies)
+    auto issue = [&](int it, int sl, bool withhold) {
         const int nn = it / p.h_v, hh = it % p.h_v, gg = hh / (p.h_v / p.h_qk);
-        if (tid == 0) {
+        if (tid == 0 && !withhold) {
             const int row0 = (sl * p.h_v + hh) * DK;
             tc::mbar_expect_tx(bar, DK * DV * 4);
 #pragma unroll
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
     __syncthreads();
     int slot = 0, nslot = 0;
     int it = next_active(blockIdx.x, &slot);
-    if (it < n_items) issue(it, slot);
+    if (it < n_items) issue(it, slot, p.test_withhold_loads != 0);
     cp_async_commit();
     uint32_t lphase = 0;  // parity of the state load being waited for
     bool fault = false;
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
         const int nx = next_active(it + gridDim.x, &nslot);  // its slot lookup overlaps the wait below
         cp_async_wait_all();
         // bounded: a load that never lands ends the kernel with a status bit, not a hang
-        if (!tc::mbar_wait(bar, lphase, kDecWaitNs)) fault = true;
+        if (!tc::mbar_wait(bar, lphase, p.wait_ns)) fault = true;
         lphase ^= 1u;
         if (__syncthreads_or(fault)) {  // this item's rows are in; the previous item's readers are done
             fault = true;
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
             sx[idx] = wv * to_f32(reinterpret_cast<const T*>(rec + C::RV)[c]);
         }
         __syncthreads();  // the raw rows are consumed, and so is each thread's state buffer
-        if (nx < n_items) issue(nx, nslot);
+        if (nx < n_items) issue(nx, nslot, false);
         cp_async_commit();
 
         const int n = it / p.h_v, h = it % p.h_v;
@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
     if (fault) {
         if (tid == 0) atomicOr(&g_status_dec, kStatusWaitTimeout);
         // give a load still in flight a last bounded chance to land before the CTA exits
-        if (tid == 0) tc::mbar_wait(bar, lphase ^ 1u, kDecWaitNs);
+        if (tid == 0) tc::mbar_wait(bar, lphase ^ 1u, p.wait_ns);
     }
 }
 

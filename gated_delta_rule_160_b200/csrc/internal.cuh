@@ -34,11 +34,13 @@ struct Params {
     // -softplus(a_raw), b, w <- sigmoid
     int prologue;
     const void* a_raw;
-    // bounded waits (tensor-core prefill): a wait longer than wait_ns is a fault; the CTA
-    // records it in the device status word, releases its tensor memory and returns
+    // bounded waits (tensor-core prefill, multi-token decode): a wait longer than wait_ns is
+    // a fault; the CTA records it in the device status word, releases its tensor memory (if
+    // any) and returns
     unsigned long long wait_ns;
-    // testing only: the prefill's producer never issues the first chunk's loads, so every
-    // wait of the CTA runs out (nothing asynchronous is in flight when it gives up)
+    // testing only: the prefill's producer never issues the first chunk's loads, and the
+    // multi-token decode never issues its first state load, so the CTA's waits run out
+    // (nothing asynchronous is in flight when it gives up)
     int test_withhold_loads;
 };
 

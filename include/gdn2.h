@@ -237,10 +237,11 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
  * since the previous gdn2_device_status on this device in *flags, and clears them. It
  * synchronises `stream` (0 = the legacy default stream); work queued on other streams is
  * covered once it has completed.
- *   GDN2_DEVICE_WAIT_TIMEOUT  a bounded wait inside the tensor-core prefill ran out (4 s):
- *                             that CTA released its tensor memory and returned without
- *                             writing its rows of o and its S_T, so the outputs of that
- *                             call are incomplete.
+ *   GDN2_DEVICE_WAIT_TIMEOUT  a bounded wait inside the tensor-core prefill or the
+ *                             multi-token decode ran out (4 s): that CTA released its
+ *                             tensor memory (prefill) and returned without writing its rows
+ *                             of o and its states, so the outputs of that call are
+ *                             incomplete.
  *   GDN2_DEVICE_BAD_SEQLENS   cu_seqlens was not 0 = c_0 <= c_1 <= ... <= c_n = T_total.
  *                             Kernels clamp every sequence to [0, T_total], so nothing is
  *                             accessed out of bounds, but the results follow the clamped
@@ -257,12 +258,13 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
 GDN2_API gdn2_status gdn2_device_status(unsigned int* flags, gdn2_stream_t stream);
 
 /*
- * Testing only: the limit of the tensor-core prefill's bounded waits for later calls from
- * any thread (wait_ns = 0 restores the default of 4 s), and, when withhold_first_load is
- * non-zero, a prefill whose producer never issues its first loads. With a short limit the
- * waits then run out, the kernel records GDN2_DEVICE_WAIT_TIMEOUT and returns, which lets a
- * test check that path without any fault: nothing asynchronous is in flight when the waits
- * give up. Not for production use.
+ * Testing only: the limit of the bounded waits of the tensor-core prefill and of the
+ * multi-token decode for later calls from any thread (wait_ns = 0 restores the default of
+ * 4 s), and, when withhold_first_load is non-zero, a prefill whose producer never issues its
+ * first loads and a multi-token decode that never issues its first state load. With a short
+ * limit the waits then run out, the kernel records GDN2_DEVICE_WAIT_TIMEOUT and returns,
+ * which lets a test check that path without any fault: nothing asynchronous is in flight
+ * when the waits give up. Not for production use.
  */
 GDN2_API void gdn2_testing_set_wait_limit(unsigned long long wait_ns, int withhold_first_load);
 
