@@ -100,6 +100,9 @@ def test_decode_multi_rejects_before_device_work(lib):
     assert call(sh, 2, 4) == 1 and b"not n_seq * n_tok" in lib.gdn2_last_error_string()
     assert call(sh, 3, 3) == 1 and b"n_slots = 3 too small" in lib.gdn2_last_error_string()
     assert call(sh, 3, 4) == 1 and b"q is NULL" in lib.gdn2_last_error_string()
+    # the pool's state rows (n_slots * h_v * dk) are TMA coordinates: int32
+    wide = _shape(g, n_seq=4, T_total=12, h_qk=32, h_v=32, dk=128, dv=128)
+    assert call(wide, 3, 1 << 20) == 2 and b"state rows" in lib.gdn2_last_error_string()
 
 
 def test_chunk_bwd_rejects_before_device_work(lib):
