@@ -66,6 +66,10 @@ constexpr int kIssuer = NS / 32;       // warp 16 issues every MMA
 constexpr int kProducer = kIssuer + 1;  // warp 17 issues every TMA load of raw chunk rows
 constexpr int NT = NS + 64;             // threads per CTA
 constexpr float kLog2e = 1.4426950408889634f;  // cumulative log-decays are kept in base 2
+// Largest |G - Gref| (base 2) for which the decay factors, times operands of order one and
+// the state's own scale, stay inside fp32's normal range with margin: a chunk whose
+// cumulative log-decay varies more than that on some channel is flagged (kStatusDecayRange)
+constexpr float kMaxFactorExp2 = 120.f;
 
 // ---- shared memory map (bytes). Tiles written by the prep are token-major, K-major, with
 // row groups outermost (LBO = 128 B, SBO = 2048 B): element (row r, channel c) at
@@ -115,7 +119,7 @@ constexpr uint32_t OFF_RAW_W = OFF_REG + 3 * kTile;   // bf16, 16 KB
 // totals [4][128]
 constexpr uint32_t OFF_SCAL = OFF_REG + 4 * kTile;
 constexpr uint32_t OFF_MBAR = OFF_SCAL + 10 * 128 * 4;
-constexpr uint32_t OFF_TSLOT = OFF_MBAR + 24 * 8;
+constexpr uint32_t OFF_TSLOT = OFF_MBAR + 24 * 8;  // tensor-memory base; +4: decay-range flag
 // fused pre-processing: 1 / max(|q|, eps) of the chunk's tokens at [0, 64), of k at [64, 128)
 constexpr uint32_t OFF_RN = OFF_TSLOT + 16;
 constexpr uint32_t SMEM_BYTES = OFF_RN + 128 * 4;
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     if (tid == 0) {
         for (int i = 0; i < kNumMbar; ++i) mbar_init(mbar(i), 1);
         fence_mbar_init();
+        *reinterpret_cast<uint32_t*>(smem + OFF_TSLOT + 4) = 0u;
     }
     if (warp == 0) tmem_alloc(sbase + OFF_TSLOT, 512);
     tc_fence_before();
@@ -497,7 +502,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         if (tid < D) {
             const int c = tid, bs = cs & 1;
             const float glast = (qtot[c] + qtot[128 + c]) + (qtot[256 + c] + qtot[384 + c]);
-            const float gref = 0.5f * (*reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c)) + glast);
+            const float g0 = *reinterpret_cast<const float*>(smem + OFF_RAW_LA + raw_off_f32(0, c));
+            const float gref = 0.5f * (g0 + glast);
+            // the factors 2^(G - Gref) reach 2^(+-|G_last - G_0| / 2) when the decays of the
+            // chunk have one sign (log_alpha <= 0): outside [2^-120, 2^120] the chunk is flagged
+            // in shared memory (nothing kept live across the chunks), posted at the end
+            if (fabsf(glast - g0) > 2.f * kMaxFactorExp2) *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT + 4) = 1u;
             fscal[c] = exp2f(cs == 0 ? gref : scal[256 + (bs ^ 1) * 128 + c] - scal[(bs ^ 1) * 128 + c]);
             fscal[128 + c] = exp2f(gref);
             scal[bs * 128 + c] = gref;
@@ -1004,6 +1014,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_status_tc, kStatusWaitTimeout);
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT + 4))
+        atomicOr(&g_status_tc, kStatusDecayRange);  // a chunk's decay factors left the safe range
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 

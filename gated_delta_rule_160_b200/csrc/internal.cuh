@@ -48,6 +48,7 @@ struct Params {
 constexpr unsigned int kStatusWaitTimeout = GDN2_DEVICE_WAIT_TIMEOUT;
 constexpr unsigned int kStatusBadSeqlens = GDN2_DEVICE_BAD_SEQLENS;
 constexpr unsigned int kStatusBadOrder = GDN2_DEVICE_BAD_ORDER;
+constexpr unsigned int kStatusDecayRange = GDN2_DEVICE_DECAY_RANGE;
 constexpr unsigned long long kDefaultWaitNs = 4000000000ull;
 
 // Pieces of the fused pre-processing, in fp32, on the special-function unit. Their errors

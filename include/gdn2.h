@@ -250,11 +250,20 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
  *                             packed-batch order (only possible when gdn2_chunk_fwd_noalloc
  *                             calls overlap on the GPU): that item was skipped, its outputs
  *                             are missing, and nothing was written out of bounds.
+ *   GDN2_DEVICE_DECAY_RANGE   in the tensor-core prefill, some key channel's cumulative
+ *                             log-decay varied by more than ~166 nats (e^(2 x 83)) within one
+ *                             64-token chunk. The kernel scales each chunk's operands by
+ *                             e^(+-(G - Gref)) around the chunk's mid-point, and beyond that
+ *                             span the factors leave fp32's range, so the results of that
+ *                             call are not reliable. (A mean log_alpha of -2.6 per token over
+ *                             a chunk reaches it; the fp32 path, taken for fp32 inputs, has
+ *                             no such limit.)
  * Returns GDN2_ERR_CUDA if the stream or the copies fail.
  */
 #define GDN2_DEVICE_WAIT_TIMEOUT 0x1u
 #define GDN2_DEVICE_BAD_SEQLENS 0x2u
 #define GDN2_DEVICE_BAD_ORDER 0x4u
+#define GDN2_DEVICE_DECAY_RANGE 0x8u
 GDN2_API gdn2_status gdn2_device_status(unsigned int* flags, gdn2_stream_t stream);
 
 /*

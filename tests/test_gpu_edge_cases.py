@@ -3,7 +3,8 @@ path (through the C ABI) against the fp64 oracle.
 
 The chunked kernel takes every decayed operand relative to the chunk's mid-point decay, so
 its fp32 factors reach e^(+-(the chunk's total log-decay) / 2): the strong-decay case puts
-about 145 nats of decay in each 64-token chunk (factors near e^72, inside fp32's range).
+about 145 nats of decay in each 64-token chunk (factors near e^72, inside fp32's range);
+past ~166 nats the kernel flags the call in the device status word.
 """
 import numpy as np
 import pytest
@@ -84,11 +85,41 @@ def test_zero_decay(g, oracle_mod):
 
 
 def test_strong_decay(g, oracle_mod):
-    """log_alpha = -2.3 per token: ~145 nats of decay across a chunk."""
+    """log_alpha = -2.3 per token: ~145 nats of decay across a chunk, inside the range of the
+    chunk kernel's factors, so the device status stays clear."""
     d = _inputs(seed=13)
     d["log_alpha"] = torch.full_like(d["log_alpha"], -2.3)
+    g.gdn2_device_status()
     o, st = _check(g, oracle_mod, d, "strong decay")
     assert torch.isfinite(o).all() and torch.isfinite(st).all()
+    assert g.gdn2_device_status() == 0
+
+
+def test_decay_beyond_the_factor_range_is_flagged(g, oracle_mod):
+    """log_alpha = -5 per token on some channels: ~320 nats across a 64-token chunk, past
+    what the chunk kernel's mid-point factors e^(+-(G - Gref)) hold in fp32. The call reports
+    GDN2_DEVICE_DECAY_RANGE; the fp32 path (fp32 inputs, sequential in the token) takes the
+    same decay exactly."""
+    d = _inputs(seed=15)
+    la = d["log_alpha"].clone()
+    la[..., :8] = -5.0
+    d["log_alpha"] = la
+    g.gdn2_device_status()
+    _run(g, d)
+    assert g.gdn2_device_status() & g.GDN2_DEVICE_DECAY_RANGE
+    d32 = dict(d)
+    for k_ in ("q", "k", "v", "b", "w"):
+        d32[k_] = d[k_].float()
+    o, st = g.gdn2_chunk_fwd(d32["q"], d32["k"], d32["v"], d32["log_alpha"], d32["b"], d32["w"], S0=d32["S0"],
+                             cu_seqlens=d32["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert g.gdn2_device_status() == 0
+    ref = oracle_on(oracle_mod, d32)
+    starts = np.concatenate([[0], np.cumsum(d32["lengths"])])
+    eo = rel_err(torch.cat([o[starts[n]:starts[n + 1], h] for (n, h) in ref]),
+                 np.concatenate([ref[key][0] for key in ref]))
+    es = rel_err(torch.stack([st[n, h] for (n, h) in ref]), np.stack([ref[key][1] for key in ref]))
+    assert eo <= TOL[torch.float32] and es <= TOL[torch.float32], (eo, es)
 
 
 def test_decay_mixed_per_channel(g, oracle_mod):
