@@ -15,6 +15,7 @@ load, importing the functions below raises.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -99,6 +100,13 @@ def _stream_handle(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _on(stream):
+    """Tensors allocated inside belong to ``stream``, the stream the call's kernels run on:
+    torch's caching allocator then hands a freed workspace (or output) only to later work
+    on that stream, never to another stream's work while the kernels still use it."""
+    return torch.cuda.stream(stream) if isinstance(stream, torch.cuda.Stream) else contextlib.nullcontext()
+
+
 def _check(status: int):
     if status != 0:
         msg = load_library().gdn2_last_error_string().decode()
@@ -143,18 +151,19 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=Non
         out_dtype = o.dtype
     shape = make_shape(q, v, n, out_dtype)
     T, h_v, dv = v.shape
-    if o is None:
-        o = torch.empty((T, h_v, dv), dtype=out_dtype, device=v.device)
-    if S_T is None and want_state:
-        S_T = torch.empty((n, h_v, q.shape[2], dv), dtype=torch.float32, device=v.device)
-    need = gdn2_chunk_fwd_workspace_size(shape, cu_seqlens is not None)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    fn = lib.gdn2_chunk_fwd_prologue if prologue else lib.gdn2_chunk_fwd
-    _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-              _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
-              _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    with _on(stream):
+        if o is None:
+            o = torch.empty((T, h_v, dv), dtype=out_dtype, device=v.device)
+        if S_T is None and want_state:
+            S_T = torch.empty((n, h_v, q.shape[2], dv), dtype=torch.float32, device=v.device)
+        need = gdn2_chunk_fwd_workspace_size(shape, cu_seqlens is not None)
+        if need and workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        fn = lib.gdn2_chunk_fwd_prologue if prologue else lib.gdn2_chunk_fwd
+        _check(fn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                  _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
+                  _ptr(workspace), ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
     return o, S_T
 
 
@@ -182,10 +191,11 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None, out_dtype
     if o is not None:
         out_dtype = o.dtype
     shape = make_shape(q, v, q.shape[0], out_dtype)
-    if o is None:
-        o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
-    _check(lib.gdn2_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                                _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream_handle(stream)))
+    with _on(stream):
+        if o is None:
+            o = torch.empty(v.shape, dtype=out_dtype, device=v.device)
+        _check(lib.gdn2_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                    _ptr(b), _ptr(w), _ptr(S), _ptr(o), _stream_handle(stream)))
     return o
 
 
@@ -205,14 +215,15 @@ def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_st
     _, _, h_v, dv = v.shape
     shape = Shape(int(N), int(N * n_tok), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v.dtype),
                   _dtype_code(out_dtype))
-    if o is None:
-        o = torch.empty((N, n_tok, h_v, dv), dtype=out_dtype, device=v.device)
-    if S_steps is None and want_steps:
-        S_steps = torch.empty((N, n_tok, h_v, dk, dv), dtype=torch.float32, device=v.device)
-    fn = lib.gdn2_decode_multi_prologue if prologue else lib.gdn2_decode_multi
-    _check(fn(ctypes.byref(shape), int(n_tok), _ptr(slots), _ptr(q), _ptr(k), _ptr(v),
-              _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
-              _ptr(o), _ptr(S_steps), _stream_handle(stream)))
+    with _on(stream):
+        if o is None:
+            o = torch.empty((N, n_tok, h_v, dv), dtype=out_dtype, device=v.device)
+        if S_steps is None and want_steps:
+            S_steps = torch.empty((N, n_tok, h_v, dk, dv), dtype=torch.float32, device=v.device)
+        fn = lib.gdn2_decode_multi_prologue if prologue else lib.gdn2_decode_multi
+        _check(fn(ctypes.byref(shape), int(n_tok), _ptr(slots), _ptr(q), _ptr(k), _ptr(v),
+                  _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(S_pool), int(S_pool.shape[0]),
+                  _ptr(o), _ptr(S_steps), _stream_handle(stream)))
     return o, S_steps
 
 
@@ -225,17 +236,19 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
     shape = make_shape(q, v, n, torch.float32)
     dev = v.device
-    f = lambda t: torch.empty(t.shape, dtype=torch.float32, device=dev)
-    dq, dk, dv, dla, db, dw = f(q), f(k), f(v), f(log_alpha), f(b), f(w)
-    dS0 = torch.empty((n, v.shape[1], q.shape[2], v.shape[2]), dtype=torch.float32, device=dev) if want_dS0 else None
-    need = int(lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(shape)))
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib.gdn2_chunk_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
-                              _ptr(S0), _ptr(cu_seqlens), _ptr(dO), _ptr(dS_T), _ptr(dq), _ptr(dk), _ptr(dv),
-                              _ptr(dla), _ptr(db), _ptr(dw), _ptr(dS0), _ptr(workspace),
-                              ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
+    with _on(stream):
+        f = lambda t: torch.empty(t.shape, dtype=torch.float32, device=dev)
+        dq, dk, dv, dla, db, dw = f(q), f(k), f(v), f(log_alpha), f(b), f(w)
+        dS0 = (torch.empty((n, v.shape[1], q.shape[2], v.shape[2]), dtype=torch.float32, device=dev)
+               if want_dS0 else None)
+        need = int(lib.gdn2_chunk_bwd_workspace_size(ctypes.byref(shape)))
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        _check(lib.gdn2_chunk_bwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b),
+                                  _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(dO), _ptr(dS_T), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(dla), _ptr(db), _ptr(dw), _ptr(dS0), _ptr(workspace),
+                                  ctypes.c_size_t(ws_bytes), _stream_handle(stream)))
     return dq, dk, dv, dla, db, dw, dS0
 
 
