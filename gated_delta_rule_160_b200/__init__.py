@@ -113,6 +113,47 @@ def _check(status: int):
         raise Gdn2Error(status, msg)
 
 
+def _expect(name, t, shape, dtype=None, device=None, optional=False):
+    """Argument check before any launch: the kernels take raw pointers and read each tensor
+    densely at the shape the call implies, so a tensor of another shape, strided, on the
+    host or of another type would be read out of bounds or misread."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} is {t.dtype}, expected {dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _expect_tokens(q, k, v, log_alpha, b, w, lead, prologue=False):
+    """q, k [*lead, Hqk, dk]; v, w [*lead, Hv, dv]; log_alpha, b [*lead, Hv, dk], one element
+    type for q, k, v, b, w (and for the decay pre-activation with the fused
+    pre-processing; log_alpha is fp32 otherwise), all on q's device."""
+    for name, t in (("q", q), ("v", v)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dim() != len(lead) + 2 or tuple(t.shape[:len(lead)]) != tuple(lead):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(lead)} + (heads, channels)")
+    h_qk, dk = q.shape[-2:]
+    h_v, dv = v.shape[-2:]
+    dt, dev = q.dtype, q.device
+    _expect("q", q, (*lead, h_qk, dk), dt, dev)
+    _expect("k", k, (*lead, h_qk, dk), dt, dev)
+    _expect("v", v, (*lead, h_v, dv), dt, dev)
+    _expect("log_alpha", log_alpha, (*lead, h_v, dk), dt if prologue else torch.float32, dev)
+    _expect("b", b, (*lead, h_v, dk), dt, dev)
+    _expect("w", w, (*lead, h_v, dv), dt, dev)
+    return h_qk, dk, h_v, dv, dev
+
+
 def _dtype_code(dt: torch.dtype) -> int:
     if dt == torch.bfloat16:
         return GDN2_BF16
@@ -149,8 +190,13 @@ def gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=Non
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
     if o is not None:
         out_dtype = o.dtype
+    T = v.shape[0] if isinstance(v, torch.Tensor) else 0
+    h_qk, dk, h_v, dv, dev = _expect_tokens(q, k, v, log_alpha, b, w, (T,), prologue)
+    _expect("S0", S0, (n, h_v, dk, dv), torch.float32, dev, optional=True)
+    _expect("cu_seqlens", cu_seqlens, (n + 1,), torch.int32, dev, optional=True)
+    _expect("o", o, (T, h_v, dv), None, dev, optional=True)
+    _expect("S_T", S_T, (n, h_v, dk, dv), torch.float32, dev, optional=True)
     shape = make_shape(q, v, n, out_dtype)
-    T, h_v, dv = v.shape
     with _on(stream):
         if o is None:
             o = torch.empty((T, h_v, dv), dtype=out_dtype, device=v.device)
@@ -177,6 +223,12 @@ def gdn2_chunk_fwd_noalloc(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n
     if o is None or S_T is None:
         raise ValueError("gdn2_chunk_fwd_noalloc writes into caller-provided o and S_T")
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
+    T = v.shape[0] if isinstance(v, torch.Tensor) else 0
+    h_qk, dk, h_v, dv, dev = _expect_tokens(q, k, v, log_alpha, b, w, (T,))
+    _expect("S0", S0, (n, h_v, dk, dv), torch.float32, dev, optional=True)
+    _expect("cu_seqlens", cu_seqlens, (n + 1,), torch.int32, dev, optional=True)
+    _expect("o", o, (T, h_v, dv), None, dev)
+    _expect("S_T", S_T, (n, h_v, dk, dv), torch.float32, dev)
     shape = make_shape(q, v, n, o.dtype)
     _check(lib.gdn2_chunk_fwd_noalloc(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                                       _ptr(b), _ptr(w), _ptr(S0), _ptr(cu_seqlens), _ptr(o), _ptr(S_T),
@@ -190,6 +242,10 @@ def gdn2_decode_step(q, k, v, log_alpha, b, w, S, o=None, stream=None, out_dtype
     lib = load_library()
     if o is not None:
         out_dtype = o.dtype
+    N = v.shape[0] if isinstance(v, torch.Tensor) else 0
+    h_qk, dk, h_v, dv, dev = _expect_tokens(q, k, v, log_alpha, b, w, (N,))
+    _expect("S", S, (N, h_v, dk, dv), torch.float32, dev)
+    _expect("o", o, (N, h_v, dv), None, dev, optional=True)
     shape = make_shape(q, v, q.shape[0], out_dtype)
     with _on(stream):
         if o is None:
@@ -211,8 +267,14 @@ def gdn2_decode_multi(q, k, v, log_alpha, b, w, S_pool, slots=None, o=None, S_st
     lib = load_library()
     if o is not None:
         out_dtype = o.dtype
-    N, n_tok, h_qk, dk = q.shape
-    _, _, h_v, dv = v.shape
+    N, n_tok = (v.shape[0], v.shape[1]) if isinstance(v, torch.Tensor) and v.dim() == 4 else (0, 0)
+    h_qk, dk, h_v, dv, dev = _expect_tokens(q, k, v, log_alpha, b, w, (N, n_tok), prologue)
+    if not isinstance(S_pool, torch.Tensor) or S_pool.dim() != 4:
+        raise ValueError("S_pool must be a CUDA tensor [n_slots, Hv, dk, dv]")
+    _expect("S_pool", S_pool, (S_pool.shape[0], h_v, dk, dv), torch.float32, dev)
+    _expect("slots", slots, (N,), torch.int32, dev, optional=True)
+    _expect("o", o, (N, n_tok, h_v, dv), None, dev, optional=True)
+    _expect("S_steps", S_steps, (N, n_tok, h_v, dk, dv), torch.float32, dev, optional=True)
     shape = Shape(int(N), int(N * n_tok), int(h_qk), int(h_v), int(dk), int(dv), _dtype_code(v.dtype),
                   _dtype_code(out_dtype))
     with _on(stream):
@@ -234,8 +296,13 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=
     (dq, dk, dv, dlog_alpha, db, dw, dS0 or None)."""
     lib = load_library()
     n = (cu_seqlens.numel() - 1) if cu_seqlens is not None else (1 if n_seq is None else int(n_seq))
+    T = v.shape[0] if isinstance(v, torch.Tensor) else 0
+    h_qk, dk, h_v, dv, dev = _expect_tokens(q, k, v, log_alpha, b, w, (T,))
+    _expect("dO", dO, (T, h_v, dv), torch.float32, dev)
+    _expect("S0", S0, (n, h_v, dk, dv), torch.float32, dev, optional=True)
+    _expect("dS_T", dS_T, (n, h_v, dk, dv), torch.float32, dev, optional=True)
+    _expect("cu_seqlens", cu_seqlens, (n + 1,), torch.int32, dev, optional=True)
     shape = make_shape(q, v, n, torch.float32)
-    dev = v.device
     with _on(stream):
         f = lambda t: torch.empty(t.shape, dtype=torch.float32, device=dev)
         dq, dk, dv, dla, db, dw = f(q), f(k), f(v), f(log_alpha), f(b), f(w)

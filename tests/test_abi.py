@@ -152,3 +152,15 @@ def test_cuda_failure_is_reported_as_cuda_error(lib):
 def test_device_status_rejects_null_flags(lib):
     assert lib.gdn2_device_status(None, None) == 1
     assert b"flags is NULL" in lib.gdn2_last_error_string()
+
+
+def test_binding_rejects_host_tensors(lib):
+    """The binding's argument checks run before any launch and need no GPU: host tensors are
+    refused with a ValueError."""
+    import torch
+    import gated_delta_rule_160_b200 as g
+    x = torch.zeros(4, 1, 64)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gdn2_chunk_fwd(x, x, x, x, x, x)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gdn2_decode_step(x, x, x, x, x, x, torch.zeros(4, 1, 64, 64))

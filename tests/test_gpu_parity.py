@@ -119,10 +119,19 @@ def test_empty_input(g):
 
 
 def test_rejects_host_memory(g):
+    """Host tensors are refused twice over: by the binding's argument checks, and by the C
+    library itself when its pointers are not device memory."""
+    import ctypes
     d = W.token_inputs(64, 1, 1, 64, 64, torch.bfloat16, "cpu", seed=1)
-    with pytest.raises(g.Gdn2Error, match="not device memory"):
-        g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"],
-                         o=torch.empty(64, 1, 64, dtype=torch.bfloat16, device="cuda"), want_state=False)
+    o = torch.empty(64, 1, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], o=o, want_state=False)
+    lib = g.load_library()
+    shape = g.make_shape(d["q"], d["v"], 1, torch.bfloat16)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    status = lib.gdn2_chunk_fwd(ctypes.byref(shape), p(d["q"]), p(d["k"]), p(d["v"]), p(d["log_alpha"]),
+                                p(d["b"]), p(d["w"]), None, None, p(o), None, None, 0, None)
+    assert status == 1 and b"not device memory" in lib.gdn2_last_error_string()
 
 
 # ------------------------------------------------------------------ decode
