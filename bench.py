@@ -93,7 +93,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc:
@@ -101,10 +101,14 @@ class ClockSampler:
             self.proc.terminate()
             self.proc.wait(timeout=5)
 
-    def summary(self):
+    def summary(self, t_from=None, t_to=None):
+        """Median SM clock, the max clock and the throttle reasons seen, over the samples that
+        arrived between host times t_from and t_to (all samples by default)."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for t, ln in self.lines:
+            if (t_from is not None and t < t_from) or (t_to is not None and t > t_to):
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -347,6 +351,19 @@ def main():
                             kernel="gdn2 chunk-forward", kernel_ms=kern_ms)
 
     o_device_run = o.cpu()  # the timed prefill's output, checked against the end-to-end path below
+
+    # The SM clock under sustained load of the same kernel: the timed region above lasts
+    # milliseconds, shorter than nvidia-smi's 50 ms sampling, so its record mostly sees the
+    # GPU idle around it. Here the step runs back to back for half a second and only the
+    # samples that arrive meanwhile count. (Not part of any timed figure.)
+    with ClockSampler(local) as loaded:
+        l_from = time.perf_counter()
+        while time.perf_counter() - l_from < 0.5:
+            for _ in range(40):
+                step()
+            torch.cuda.synchronize()
+        l_to = time.perf_counter()
+    clocks_loaded = loaded.summary(l_from + 0.06, l_to)
 
     # ---------------- prefill with the fused pre-processing (raw projections in)
     gen = torch.Generator(device=dev).manual_seed(wl.seed + 17)
@@ -638,6 +655,7 @@ def main():
             "cpu_baseline": base,
             "decode": decode,
             "clocks": clocks.summary(),
+            "clocks_loaded": clocks_loaded,
             "gpu_launches": args.steps,
         }
         print(json.dumps(line), flush=True)
