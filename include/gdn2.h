@@ -134,6 +134,9 @@ GDN2_API gdn2_status gdn2_decode_step(const gdn2_shape* shape,
  *   token, so that a caller that accepts only the first j drafted tokens can put back the
  *   state after token j - 1 (S_pool itself always ends after all n_tok tokens).
  * Errors as for the other calls; slot values are only checked on the device (skipped).
+ * GDN2_ERR_UNSUPPORTED if n_slots * h_v * dk exceeds 2^31 - 1 (the pool's state rows are
+ * addressed as 32-bit coordinates). With n_tok > 1 (or S_steps given) each state is
+ * loaded by TMA and its wait is bounded like the prefill's (GDN2_DEVICE_WAIT_TIMEOUT).
  */
 #define GDN2_DECODE_MAX_TOKENS 8
 GDN2_API gdn2_status gdn2_decode_multi(const gdn2_shape* shape, int n_tok, const int32_t* slots,
