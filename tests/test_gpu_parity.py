@@ -209,6 +209,24 @@ def test_full_size_sampled(g, oracle_mod, name, seqs, qk_heads):
     _compare(g, oracle_mod, d, wl.dtype, seqs=seqs, qk_heads=qk_heads, label=name)
 
 
+@pytest.mark.parametrize("name", ["prefill_b8_h16_t4096", "grouped_b2_qk16_v32_t32768", "varlen_64seq_h16"])
+def test_full_size_every_pair_against_the_fp32_path(g, name):
+    """Every output of the tensor-core prefill at full size, against the fp32 per-token
+    kernel (itself pinned to the oracle at 1e-4) run on the same values widened to fp32: the
+    chunked and the sequential form of the recurrence, within the bf16 bound."""
+    wl = W.WORKLOADS[name]
+    d = W.prefill_inputs(wl, "cuda")
+    args = dict(S0=d["S0"], cu_seqlens=d["cu_seqlens"], n_seq=d["n_seq"])
+    o, st = g.gdn2_chunk_fwd(*(d[k_] for k_ in ("q", "k", "v", "log_alpha", "b", "w")), **args)
+    o32, st32 = g.gdn2_chunk_fwd(*(d[k_].float() for k_ in ("q", "k", "v", "log_alpha", "b", "w")), **args)
+    torch.cuda.synchronize()
+    assert g.gdn2_device_status() == 0
+    eo = rel_err(o, o32.double().cpu().numpy())
+    es = rel_err(st, st32.double().cpu().numpy())
+    print(f"{name} against the fp32 path, every pair: o err {eo:.3e}, S_T err {es:.3e}")
+    assert eo <= TOL[torch.bfloat16] and es <= TOL[torch.bfloat16], (eo, es)
+
+
 def test_decode_full_size_sampled(g, oracle_mod):
     """All 256 x 32 states through all 512 steps on the GPU; the oracle replays sampled
     (sequence, head) pairs as 512-token sequences."""
