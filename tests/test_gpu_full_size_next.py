@@ -132,3 +132,53 @@ def test_serving_decode_full_size_sampled(g):
     es = rel_err(torch.stack(s_got), np.stack(s_ref))
     print(f"serving decode full size: o err {eo:.3e}, S err {es:.3e} (tol {tol})")
     assert eo <= tol and es <= tol
+
+
+def test_prologue_full_size_every_pair_against_the_fp32_path(g):
+    """Every output of gdn2_chunk_fwd_prologue at full size, against the fp32 per-token kernel
+    given the activations written out in torch (fp32): q / max(|q|, eps), k likewise,
+    -softplus(a), sigmoid(b), sigmoid(w)."""
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, "cuda")
+    T_all = int(sum(d["lengths"]))
+    gen = torch.Generator(device="cuda").manual_seed(wl.seed + 17)
+    rn = lambda *shp: torch.randn(*shp, generator=gen, device="cuda").to(wl.dtype)
+    raw = dict(q=rn(T_all, wl.h_qk, wl.dk), k=rn(T_all, wl.h_qk, wl.dk), a=rn(T_all, wl.h_v, wl.dk),
+               b=rn(T_all, wl.h_v, wl.dk), w=rn(T_all, wl.h_v, wl.dv))
+    o, st = g.gdn2_chunk_fwd(raw["q"], raw["k"], d["v"], raw["a"], raw["b"], raw["w"], S0=d["S0"],
+                             n_seq=d["n_seq"], prologue=True)
+    unit = lambda x: x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+    act = dict(q=unit(raw["q"].float()), k=unit(raw["k"].float()), v=d["v"].float(),
+               log_alpha=-torch.nn.functional.softplus(raw["a"].float()), b=torch.sigmoid(raw["b"].float()),
+               w=torch.sigmoid(raw["w"].float()))
+    o32, st32 = g.gdn2_chunk_fwd(*(act[key] for key in ("q", "k", "v", "log_alpha", "b", "w")), S0=d["S0"],
+                                 n_seq=d["n_seq"])
+    torch.cuda.synchronize()
+    eo = rel_err(o, o32.double().cpu().numpy())
+    es = rel_err(st, st32.double().cpu().numpy())
+    print(f"prologue full size, every pair against the fp32 path: o err {eo:.3e}, S_T err {es:.3e}")
+    assert eo <= TOL[torch.bfloat16] and es <= TOL[torch.bfloat16], (eo, es)
+
+
+def test_serving_decode_full_size_every_state_against_the_prefill(g):
+    """gdn2_decode_multi on all 256 x 32 states of the serving workload (4 tokens, states at
+    seeded-random slots of a 512-state pool) equals, for every state, the fp32 prefill of the
+    same 4 tokens started from that state."""
+    wl = W.WORKLOADS[DECODE]
+    N, n_tok = wl.n_seq, 4
+    pool = torch.zeros((2 * N, wl.h_v, wl.dk, wl.dv), dtype=torch.float32, device="cuda")
+    perm = torch.randperm(2 * N, generator=torch.Generator().manual_seed(wl.seed))[:N]
+    S_init = W.decode_state(wl, "cuda")
+    pool[perm.to("cuda")] = S_init
+    slots = perm.to(torch.int32).to("cuda")
+    t_ = W.token_inputs(N * n_tok, wl.h_qk, wl.h_v, wl.dk, wl.dv, wl.dtype, "cuda", wl.seed * 7919)
+    x = {key: t.view(N, n_tok, *t.shape[1:]) for key, t in t_.items()}
+    o, _ = g.gdn2_decode_multi(*(x[key] for key in ("q", "k", "v", "log_alpha", "b", "w")), pool, slots=slots)
+    f = {key: t_[key].float() for key in ("q", "k", "v", "log_alpha", "b", "w")}
+    o_pre, S_pre = g.gdn2_chunk_fwd(*(f[key] for key in ("q", "k", "v", "log_alpha", "b", "w")), S0=S_init,
+                                    n_seq=N)
+    torch.cuda.synchronize()
+    eo = rel_err(o.reshape(N * n_tok, wl.h_v, wl.dv), o_pre.double().cpu().numpy())
+    es = rel_err(pool[perm.to("cuda")], S_pre.double().cpu().numpy())
+    print(f"serving decode full size, every state against the prefill: o err {eo:.3e}, S err {es:.3e}")
+    assert eo <= TOL[torch.float32] and es <= TOL[torch.float32], (eo, es)
