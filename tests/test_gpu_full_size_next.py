@@ -182,3 +182,44 @@ def test_serving_decode_full_size_every_state_against_the_prefill(g):
     es = rel_err(pool[perm.to("cuda")], S_pre.double().cpu().numpy())
     print(f"serving decode full size, every state against the prefill: o err {eo:.3e}, S err {es:.3e}")
     assert eo <= TOL[torch.float32] and es <= TOL[torch.float32], (eo, es)
+
+
+def test_backward_full_size_directional_derivatives(g):
+    """The gradients of the full-size backward over every (sequence, head) pair at once: o is
+    linear in S0, in v, in w and in q, so for a random direction delta the central difference
+    [L(x + delta) - L(x - delta)] / 2 of L = sum(o * dO) equals <dL/dx, delta> exactly (up to
+    rounding), whatever delta's size; for k, b and log_alpha, extrapolated central differences
+    at small steps. L is taken with the fp32 forward kernel on the same input values."""
+    wl = W.WORKLOADS[PREFILL]
+    d = W.prefill_inputs(wl, "cuda")
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+    S0 = W.state_input(wl.n_seq, wl.h_v, wl.dk, wl.dv, 0.05, "cuda", seed=wl.seed + 5)
+    gen = torch.Generator(device="cuda").manual_seed(wl.seed + 29)
+    dO = torch.randn(d["v"].shape, generator=gen, device="cuda")
+    dq, dk, dv, dla, db, dw, dS0 = g.gdn2_chunk_bwd(*(d[k_] for k_ in names), dO, S0=S0, n_seq=wl.n_seq)
+    f32 = {k_: d[k_].float() for k_ in names}
+
+    def loss(**over):
+        x = dict(f32, **{k_: v_ for k_, v_ in over.items() if k_ != "S0"})
+        o, _ = g.gdn2_chunk_fwd(*(x[k_] for k_ in names), S0=over.get("S0", S0), n_seq=wl.n_seq, want_state=False)
+        return float((o.double() * dO.double()).sum())
+
+    checks = []
+    for name, grad, base in (("S0", dS0, S0), ("v", dv, f32["v"]), ("q", dq, f32["q"]), ("w", dw, f32["w"])):
+        delta = torch.randn(base.shape, generator=gen, device="cuda") * base.abs().mean()
+        fd = (loss(**{name: base + delta}) - loss(**{name: base - delta})) / 2.0
+        an = float((grad.double() * delta.double()).sum())
+        checks.append((name, fd, an, abs(fd - an) / abs(an)))
+    # k, b and log_alpha enter non-linearly: central differences at steps h and 2h, combined
+    # (Richardson) so that the h^2 term cancels, leave O(h^4)
+    for name, grad, base, h in (("k", dk, f32["k"], 1e-2), ("b", db, f32["b"], 1e-2),
+                                ("log_alpha", dla, f32["log_alpha"], 1e-2)):
+        delta = torch.randn(base.shape, generator=gen, device="cuda") * base.abs().mean()
+        cd = lambda s_: (loss(**{name: base + s_ * delta}) - loss(**{name: base - s_ * delta})) / (2.0 * s_)
+        fd = (4.0 * cd(h) - cd(2.0 * h)) / 3.0
+        an = float((grad.double() * delta.double()).sum())
+        checks.append((name, fd, an, abs(fd - an) / abs(an)))
+    for name, fd, an, rel in checks:
+        print(f"backward full size, directional {name}: difference {fd:.6e}, gradient {an:.6e}, rel {rel:.2e}")
+    # the linear ones to rounding; the others to the extrapolation's remainder
+    assert all(rel <= (1e-4 if name in ("S0", "v", "q", "w") else 2e-3) for name, *_, rel in checks), checks
