@@ -34,7 +34,7 @@ ABI_FUNCTIONS = ("gdn2_chunk_fwd_workspace_size", "gdn2_chunk_fwd", "gdn2_chunk_
                  "gdn2_version")
 # bits of the device status word (gdn2_device_status)
 GDN2_DEVICE_WAIT_TIMEOUT, GDN2_DEVICE_BAD_SEQLENS, GDN2_DEVICE_BAD_ORDER = 0x1, 0x2, 0x4
-GDN2_DEVICE_DECAY_RANGE = 0x8
+GDN2_DEVICE_DECAY_RANGE = 0x8  # a pair was recomputed token by token (valid, slower)
 
 
 class Gdn2Error(RuntimeError):

@@ -208,6 +208,154 @@ __device__ __forceinline__ void store8_bf16(uint8_t* smem, uint32_t off, const f
 template <typename TO>
 constexpr bool kTmaStoreO = sizeof(TO) == 4;  // the o tensor map is fp32
 
+// ---- token-by-token recomputation of one (sequence, value head)
+// A CTA whose decay left the chunk frame's range (kMaxFactorExp2) finishes its chunk walk
+// (results unusable, S_T not written) and then runs the recurrence itself over the whole
+// sequence in fp32, from S0, overwriting that pair's o and writing S_T: per token, decay
+// the state by alpha, read r = S'^T k and p = S'^T q, edit S = S' - (b k) r^T + k (w v)^T,
+// and emit o = p - (q.(b k)) r + (q.k) (w v), which is the updated state's read by q.
+// The 512 SIMT threads hold the state in registers: warp w takes value column
+// 32 (w / 4) + lane and key rows 32 (w % 4) .. + 31; the four partial reads of a column
+// are added through shared memory after one barrier per token. Inputs are staged 16
+// tokens at a time in shared memory as fp32, with the fused pre-processing applied for
+// kPro (L2 norms of q and k, alpha = e^(-softplus(a)) = sigmoid(-a), sigmoid gates).
+constexpr int kRedoStage = 16;
+struct RedoSmem {
+    float k[kRedoStage][D];
+    float q[kRedoStage][D];
+    float a[kRedoStage][D];  // alpha
+    float e[kRedoStage][D];  // b (.) k
+    float x[kRedoStage][D];  // w (.) v
+    float qe[kRedoStage];    // q . (b (.) k)
+    float qk[kRedoStage];    // q . k
+    float red[2][2][4][D];   // [token parity][r | p][row quarter][value column]
+};
+static_assert(sizeof(RedoSmem) <= OFF_MBAR, "recomputation staging overlaps the barriers");
+
+template <typename TO, bool kPro>
+__device__ __forceinline__ void redo_tokens(const Params& p, int h, int g, int t0, int t1, size_t soff,
+                                         uint8_t* smem_raw, int tid) {
+    RedoSmem& sm = *reinterpret_cast<RedoSmem*>(smem_raw);
+    const int warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;
+    const int col = 32 * (warp >> 2) + lane;
+    const int row0 = 32 * quarter;
+    const __nv_bfloat16* qp = static_cast<const __nv_bfloat16*>(p.q);
+    const __nv_bfloat16* kp = static_cast<const __nv_bfloat16*>(p.k);
+    const __nv_bfloat16* vp = static_cast<const __nv_bfloat16*>(p.v);
+    const __nv_bfloat16* bp = static_cast<const __nv_bfloat16*>(p.b);
+    const __nv_bfloat16* wp = static_cast<const __nv_bfloat16*>(p.w);
+    const __nv_bfloat16* ap = static_cast<const __nv_bfloat16*>(p.a_raw);
+    TO* op = static_cast<TO*>(p.o);
+
+    float s[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) s[i] = p.S0 ? p.S0[soff + (size_t)(row0 + i) * D + col] : 0.f;
+
+    for (int base = t0; base < t1; base += kRedoStage) {
+        const int nt = min(kRedoStage, t1 - base);
+        bar_sync_1<NS>();  // the previous stage is consumed
+        for (int idx = tid; idx < nt * D; idx += NS) {
+            const int tt = idx / D, c = idx % D;
+            const size_t t = (size_t)(base + tt);
+            const size_t oqk = (t * p.h_qk + g) * D + c, ov = (t * p.h_v + h) * D + c;
+            float bv = to_f32(bp[ov]), wv = to_f32(wp[ov]);
+            float av;
+            if (kPro) {
+                av = sigmoid_f(-to_f32(ap[ov]));
+                bv = sigmoid_f(bv);
+                wv = sigmoid_f(wv);
+            } else {
+                av = expf(p.log_alpha[ov]);
+            }
+            sm.k[tt][c] = to_f32(kp[oqk]);
+            sm.q[tt][c] = to_f32(qp[oqk]);
+            sm.a[tt][c] = av;
+            sm.e[tt][c] = bv;  // times k below
+            sm.x[tt][c] = wv * to_f32(vp[ov]);
+        }
+        bar_sync_1<NS>();
+        if (warp < nt) {  // warp tt: q and k normalised (kPro), b (.) k, q . e and q . k
+            const int tt = warp;
+            float kv[4], qv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                kv[j] = sm.k[tt][lane + 32 * j];
+                qv[j] = sm.q[tt][lane + 32 * j];
+            }
+            if (kPro) {
+                float sk = 0.f, sq = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    sk = fmaf(kv[j], kv[j], sk);
+                    sq = fmaf(qv[j], qv[j], sq);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                }
+                const float rk = rsqrtf(fmaxf(sk, kL2NormEps * kL2NormEps));
+                const float rq = rsqrtf(fmaxf(sq, kL2NormEps * kL2NormEps));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    kv[j] *= rk;
+                    qv[j] *= rq;
+                    sm.k[tt][lane + 32 * j] = kv[j];
+                    sm.q[tt][lane + 32 * j] = qv[j];
+                }
+            }
+            float d1 = 0.f, d2 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float e = sm.e[tt][lane + 32 * j] * kv[j];
+                sm.e[tt][lane + 32 * j] = e;
+                d1 = fmaf(qv[j], e, d1);
+                d2 = fmaf(qv[j], kv[j], d2);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                d1 += __shfl_xor_sync(0xffffffffu, d1, o);
+                d2 += __shfl_xor_sync(0xffffffffu, d2, o);
+            }
+            if (lane == 0) {
+                sm.qe[tt] = d1;
+                sm.qk[tt] = d2;
+            }
+        }
+        bar_sync_1<NS>();
+        for (int tt = 0; tt < nt; ++tt) {
+            float r = 0.f, pq = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                s[i] *= sm.a[tt][row0 + i];
+                r = fmaf(sm.k[tt][row0 + i], s[i], r);
+                pq = fmaf(sm.q[tt][row0 + i], s[i], pq);
+            }
+            const int par = tt & 1;
+            sm.red[par][0][quarter][col] = r;
+            sm.red[par][1][quarter][col] = pq;
+            bar_sync_1<NS>();  // (a buffer is rewritten two tokens later, after the next barrier)
+            r = 0.f;
+            pq = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                r += sm.red[par][0][w][col];
+                pq += sm.red[par][1][w][col];
+            }
+            const float x = sm.x[tt][col];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[i] = fmaf(sm.k[tt][row0 + i], x, fmaf(-sm.e[tt][row0 + i], r, s[i]));
+            if (quarter == (tt & 3))
+                op[((size_t)(base + tt) * p.h_v + h) * D + col] = from_f32<TO>(pq - sm.qe[tt] * r + sm.qk[tt] * x);
+        }
+    }
+    if (p.S_T) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p.S_T[soff + (size_t)(row0 + i) * D + col] = s[i];
+    }
+}
+
 // kPro: fused pre-processing. The raw q, k are L2-normalised per token (norms over the 128
 // channels, reduced across the eight warps of a token through shared memory), log_alpha is
 // -softplus of the bf16 decay pre-activation (staged as a bf16 tile beside the cumulative
@@ -986,20 +1134,30 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
         }
         tc_fence_before();
     }
+    // redo: some chunk's decay left the frame's range (the flag is set before a barrier the
+    // SIMT warps have all passed); this pair is then recomputed token by token below
+    bool redo = false;
     if (warp < kIssuer) {
         bar_sync_1<NS>();
+        redo = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT + 4) != 0u;
         const int tcl = t0 + (nchunks - 1) * CH;
         if (kTmaStoreO<TO> && !fault && t1 - tcl == CH && tid == 0) {  // the last chunk's staged o
             tma_store_3d(&maps.o, sbase + OFF_OST0, 0, h, tcl);
             tma_store_3d(&maps.o, sbase + OFF_OST1, 0, h, tcl + CH / 2);
             bulk_commit();
         }
-        // the staged o tile must be read out before shared memory is released or rewritten
-        if (tid == 0) bulk_wait_read0();
+        // the staged o tile must be read out before shared memory is released or rewritten,
+        // and, when o is recomputed, written out before the recomputation's stores
+        if (tid == 0) {
+            if (redo) bulk_wait_all0();
+            else bulk_wait_read0();
+        }
         if (!fault) fault = !mbar_wait(mbar(MB_45), (uint32_t)((nchunks - 1) & 1), kWaitNs);
+        fault = bar_or_1<NS>(fault);  // one decision for all SIMT warps
+        redo = redo && !fault;
     }
 
-    if (!fault && p.S_T && warp < kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
+    if (!fault && !redo && p.S_T && warp < kIssuer) {  // S_T[c][m] = exp(G_last - Gref) (.) U[m][c]
         const int buf = (nchunks - 1) & 1;
         tc_fence_after();
         const int cb = 32 * cp;
@@ -1014,9 +1172,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
     if (fault && (tid == 0 || tid == NS || tid == NS + 32)) atomicOr(&g_status_tc, kStatusWaitTimeout);
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *reinterpret_cast<volatile uint32_t*>(smem + OFF_TSLOT + 4))
-        atomicOr(&g_status_tc, kStatusDecayRange);  // a chunk's decay factors left the safe range
+    if (tid == 0 && redo) atomicOr(&g_status_tc, kStatusDecayRange);  // recomputed below
     if (warp == 0) tmem_dealloc(tmem, 512);
+    if (redo) redo_tokens<TO, kPro>(p, h, g, t0, t1, soff, smem, tid);  // SIMT warps only
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

@@ -299,6 +299,11 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int x, int y, 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the shared memory read by all committed bulk stores of this thread may be reused.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until all committed bulk stores of this thread have written global memory, then
+// order those (async-proxy) writes before this thread's later generic accesses.
+__device__ __forceinline__ void bulk_wait_all0() {
+    asm volatile("cp.async.bulk.wait_group 0;\n\tfence.proxy.async.global;" ::: "memory");
+}
 
 // Prefetch the cache line holding ptr into L2.
 __device__ __forceinline__ void prefetch_line_l2(const void* ptr) {

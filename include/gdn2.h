@@ -94,7 +94,8 @@ GDN2_API size_t gdn2_chunk_fwd_workspace_size(const gdn2_shape* shape, int varle
  * token). Sequences are packed by cu_seqlens; with cu_seqlens == NULL, T_total must be a
  * multiple of n_seq and sequence n is tokens [n*T, (n+1)*T), T = T_total / n_seq.
  * S0 == NULL starts every sequence from a zero state. S_T == NULL skips the final state.
- * A zero-length sequence writes S_T = S0 (or 0) and no output.
+ * S_T may be S0 itself (the states are then updated in place); no other output may overlap
+ * an input. A zero-length sequence writes S_T = S0 (or 0) and no output.
  * workspace: device memory of at least gdn2_chunk_fwd_workspace_size() bytes, 256-byte
  * aligned, owned by the caller, reused freely after the call's work completes; may be
  * NULL when that size is 0.
@@ -257,10 +258,12 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
  *                             log-decay varied by more than ~166 nats (e^(2 x 83)) within one
  *                             64-token chunk. The kernel scales each chunk's operands by
  *                             e^(+-(G - Gref)) around the chunk's mid-point, and beyond that
- *                             span the factors leave fp32's range, so the results of that
- *                             call are not reliable. (A mean log_alpha of -2.6 per token over
- *                             a chunk reaches it; the fp32 path, taken for fp32 inputs, has
- *                             no such limit.)
+ *                             span the factors leave fp32's range; the CTA of that (sequence,
+ *                             head) then recomputes its o and S_T token by token in fp32
+ *                             within the same launch, from S0 (which it has not overwritten),
+ *                             so the results are valid. The bit says that this slower route
+ *                             ran (~1 us per token for each such pair). A mean log_alpha of
+ *                             -2.6 per token over a chunk reaches it.
  * Returns GDN2_ERR_CUDA if the stream or the copies fail.
  */
 #define GDN2_DEVICE_WAIT_TIMEOUT 0x1u

@@ -54,6 +54,30 @@ def test_chunk_prologue_matches_oracle(g):
     torch.testing.assert_close(st[3], S0[3], rtol=0, atol=0)  # the empty sequence
 
 
+def test_chunk_prologue_decay_beyond_range_is_recomputed(g):
+    """A decay pre-activation of +6 on eight channels of one (sequence, head) gives
+    log_alpha = -softplus(6) ~ -6 per token, ~380 nats across a chunk: past the tensor-core
+    kernel's range, so that pair is recomputed token by token in fp32 (the pre-processing
+    included) and matches the oracle to the fp32 bound; the rest keep the bf16 bound."""
+    lens = [200, 64, 131]
+    T = sum(lens)
+    d = _raw(T, 2, 4, seed=44)
+    a = d["a"].clone()
+    a[264:395, 3, 40:48] = 6.0  # sequence 2, value head 3
+    d["a"] = a
+    S0 = W.state_input(len(lens), 4, D, D, 0.05, "cuda", seed=44)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    g.gdn2_device_status()
+    o, st = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["a"], d["b"], d["w"], S0=S0, cu_seqlens=cu, prologue=True)
+    torch.cuda.synchronize()
+    assert g.gdn2_device_status() & g.GDN2_DEVICE_DECAY_RANGE
+    o_ref, st_ref = _oracle(d, S0, cu.cpu())
+    eo, es = rel_err(o[264:, 3], o_ref[264:, 3]), rel_err(st[2, 3], st_ref[2, 3])
+    print(f"recomputed pair: o err {eo:.3e}, S_T err {es:.3e} (tol {TOL[torch.float32]})")
+    assert eo <= TOL[torch.float32] and es <= TOL[torch.float32]
+    assert rel_err(o, o_ref) <= TOL[torch.bfloat16] and rel_err(st, st_ref) <= TOL[torch.bfloat16]
+
+
 def test_decode_prologue_matches_oracle(g):
     N, n_tok, H, n_slots = 4, 3, 2, 6
     slots = [5, 0, 3, 1]
