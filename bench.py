@@ -145,8 +145,8 @@ def prefill_bytes(wl, lengths, o_bytes=None) -> int:
     """Algorithmic bytes of one chunk-forward: every input read once, o and S_T written once
     (S0 read once when given); q and k are counted once per query/key head (value heads in a
     group share them). o_bytes is the size of one output element: by default that of the
-    input dtype, which is the survey's count (2048 B per token and head for bf16 inputs,
-    d = 128); the kernel writes o in fp32 (o_bytes = 4, 2304 B)."""
+    input dtype, the algorithmic count (2048 B per token and head for bf16 inputs, d = 128);
+    the kernel writes o in fp32 (o_bytes = 4, 2304 B)."""
     es = torch.finfo(wl.dtype).bits // 8
     ob = es if o_bytes is None else o_bytes
     T = int(sum(lengths))
@@ -159,7 +159,7 @@ def prefill_bytes(wl, lengths, o_bytes=None) -> int:
 
 def hbm_roofline(nbytes: int, nbytes_f32o: int, ms: float, hbm: float, peak_src: str, traffic, **extra):
     """The HBM roofline of one chunk-forward launch of ms milliseconds: achieved = the
-    survey's algorithmic bytes / time; the same with o counted as the fp32 it is written in
+    algorithmic bytes / time; the same with o counted as the fp32 it is written in
     alongside."""
     ach = nbytes / (ms / 1000.0) / 1e9
     ach32 = nbytes_f32o / (ms / 1000.0) / 1e9
@@ -384,6 +384,30 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     pms = max_over_ranks(e0.elapsed_time(e1) / PROLOGUE_TIMED_STEPS, world)
+
+    # For comparison only: the same pre-processing left to the caller as torch elementwise
+    # ops, then the plain kernel on the activated inputs.
+    def ustep():
+        with torch.cuda.stream(stream):
+            nf = torch.nn.functional
+            qn = nf.normalize(raw["q"].float(), dim=-1, eps=1e-12).to(wl.dtype)
+            kn = nf.normalize(raw["k"].float(), dim=-1, eps=1e-12).to(wl.dtype)
+            la = nf.softplus(raw["a"].float()).neg_()
+            bs = torch.sigmoid(raw["b"].float()).to(wl.dtype)
+            ws = torch.sigmoid(raw["w"].float()).to(wl.dtype)
+        G.gdn2_chunk_fwd(qn, kn, d["v"], la, bs, ws, S0=d["S0"], n_seq=d["n_seq"], o=o, S_T=S_T, stream=stream)
+    for _ in range(3):
+        ustep()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(PROLOGUE_TIMED_STEPS):
+        ustep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ums = max_over_ranks(e0.elapsed_time(e1) / PROLOGUE_TIMED_STEPS, world)
+
     pbytes = prologue_bytes(wl, d["lengths"])
     pach = pbytes / (pms / 1000.0) / 1e9
     prologue = {"metric": "GDN-2 chunk-fwd tokens/s, fused pre-processing", "value": world * T_all / (pms / 1000.0),
@@ -391,7 +415,9 @@ def main():
                 "config": {"workload": f"{PREFILL} from raw projections (bf16 decay pre-activation)"},
                 "roofline": {"bound": "hbm", "achieved": pach, "peak": hbm, "unit": "GB/s", "frac": pach / hbm,
                              "traffic": recorded_traffic("chunk_tc_prologue_prefill_b8_h16_t4096"),
-                             "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": pbytes}}
+                             "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": pbytes},
+                "unfused_ms_per_step": ums,
+                "unfused": "the same pre-processing as torch elementwise ops, then gdn2_chunk_fwd (comparison)"}
     del raw
 
     # ---------------- backward (gradients of sum(o * dO)), same workload

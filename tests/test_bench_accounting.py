@@ -25,7 +25,7 @@ def bench():
 def test_prefill_bytes_headline(bench):
     wl = W.WORKLOADS["prefill_b8_h16_t4096"]
     tokens = 8 * 4096
-    # the survey's count: per token, q, k bf16 on 16 query/key heads; v, w, b bf16, log_alpha
+    # the algorithmic count: per token, q, k bf16 on 16 query/key heads; v, w, b bf16, log_alpha
     # fp32 and o at the input dtype (bf16) on 16 value heads -- 2048 B per token and head;
     # plus S_T written once (S0 is zero and not read)
     per_token = 16 * (128 * 2 + 128 * 2) + 16 * (128 * 2 + 128 * 2 + 128 * 2 + 128 * 4 + 128 * 2)
@@ -43,7 +43,7 @@ def test_prefill_bytes_grouped_counts_qk_once_per_query_key_head(bench):
     per_token = 16 * 512 + 32 * 1536           # q, k per query/key head; the rest per value head
     state = 2 * 32 * 128 * 128 * 4
     assert bench.prefill_bytes(wl, [32768] * 2) == tokens * per_token + 2 * state  # S0 read, S_T written
-    # the survey's 1792 B per token and value head (q and k shared by two value heads)
+    # 1792 B per token and value head (q and k shared by two value heads)
     assert per_token == 32 * 1792
 
 

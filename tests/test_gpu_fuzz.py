@@ -1,6 +1,6 @@
 """Seeded random configurations through the C ABI against the fp64 oracle: dtypes, key and
 value widths, head groupings, ragged and empty packed sequences, initial states; decode over
-a slot pool with inactive slots and 1..8 tokens; and the gradients. Small sizes, so the
+a slot pool with inactive slots and 1..8 tokens; bursts of strong decay; and the gradients. Small sizes, so the
 oracle sees whole tensors."""
 import numpy as np
 import pytest
@@ -50,6 +50,42 @@ def test_fuzz_chunk_fwd(g, seed):
     eo, es = rel_err(o, o_ref), rel_err(st, s_ref)
     print(f"fuzz chunk {c}: o {eo:.2e}, S_T {es:.2e}")
     assert eo <= tol and es <= tol, c
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_fuzz_chunk_fwd_decay_spikes(g, seed):
+    """The tensor-core shape with bursts of strong decay: random (token range, value head,
+    channel) blocks at -2 .. -9 per token and single tokens at -20 .. -120, so that some
+    (sequence, head) pairs leave the chunk frame's range (and are recomputed token by token)
+    and others stay just inside it. Every pair is checked against the oracle."""
+    rng = np.random.default_rng(3000 + seed)
+    h_qk = int(rng.choice([1, 2]))
+    h_v = h_qk * int(rng.choice([1, 2]))
+    lens = [int(x) for x in rng.choice([1, 63, 64, 65, 130, 200], size=int(rng.integers(1, 4)))]
+    T = sum(lens)
+    d = W.token_inputs(T, h_qk, h_v, 128, 128, torch.bfloat16, "cuda", seed=seed)
+    la = d["log_alpha"].clone()
+    for _ in range(int(rng.integers(1, 4))):
+        t0 = int(rng.integers(0, T))
+        t1 = min(T, t0 + int(rng.integers(8, 80)))
+        c0 = int(rng.integers(0, 120))
+        la[t0:t1, int(rng.integers(0, h_v)), c0:c0 + int(rng.integers(1, 9))] = -float(rng.uniform(2.0, 9.0))
+    for _ in range(int(rng.integers(0, 4))):
+        la[int(rng.integers(0, T)), int(rng.integers(0, h_v)), int(rng.integers(0, 128))] = -float(rng.uniform(20, 120))
+    d["log_alpha"] = la
+    S0 = W.state_input(len(lens), h_v, 128, 128, 0.05, "cuda", seed=seed)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device="cuda")
+    g.gdn2_device_status()
+    o, st = g.gdn2_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["b"], d["w"], S0=S0, cu_seqlens=cu)
+    torch.cuda.synchronize()
+    flags = g.gdn2_device_status()
+    assert flags & ~g.GDN2_DEVICE_DECAY_RANGE == 0
+    o_ref, s_ref = oracle.fwd_ref(*(d[k].cpu() for k in ("q", "k", "v", "log_alpha", "b", "w")),
+                                  S0=S0.cpu(), cu_seqlens=cu.cpu())
+    eo, es = rel_err(o, o_ref), rel_err(st, s_ref)
+    print(f"fuzz decay spikes {seed}: lens {lens}, heads {h_qk}/{h_v}, recomputed {bool(flags)}: "
+          f"o {eo:.2e}, S_T {es:.2e}")
+    assert eo <= TOL[torch.bfloat16] and es <= TOL[torch.bfloat16]
 
 
 @pytest.mark.parametrize("seed", range(8))
