@@ -262,7 +262,8 @@ GDN2_API gdn2_status gdn2_chunk_fwd_noalloc(const gdn2_shape* shape,
  *                             head) then recomputes its o and S_T token by token in fp32
  *                             within the same launch, from S0 (which it has not overwritten),
  *                             so the results are valid. The bit says that this slower route
- *                             ran (~1 us per token for each such pair). A mean log_alpha of
+ *                             ran (~1.1 us per token of the longest such pair, measured on
+ *                             B200: 5.0 ms for 4096 tokens against 0.57 ms). A mean log_alpha of
  *                             -2.6 per token over a chunk reaches it.
  * Returns GDN2_ERR_CUDA if the stream or the copies fail.
  */
