@@ -54,6 +54,9 @@ gdn2_status check_shape(const gdn2_shape* sh) {
     if (sh->h_v % sh->h_qk != 0)
         return fail(GDN2_ERR_INVALID_ARG, "h_v = %d is not a multiple of h_qk = %d", sh->h_v, sh->h_qk);
     if (sh->h_v > 65535) return fail(GDN2_ERR_UNSUPPORTED, "h_v = %d above 65535", sh->h_v);
+    if ((long long)sh->n_seq * sh->h_v > 0x7fffffffLL)  // one CTA per (sequence, value head)
+        return fail(GDN2_ERR_UNSUPPORTED, "n_seq * h_v = %lld (sequence, head) pairs above 2^31 - 1",
+                    (long long)sh->n_seq * sh->h_v);
     if (sh->dtype != GDN2_F32 && sh->dtype != GDN2_BF16)
         return fail(GDN2_ERR_INVALID_ARG, "unknown dtype %d", (int)sh->dtype);
     if (sh->o_dtype != GDN2_F32 && sh->o_dtype != GDN2_BF16)

@@ -43,7 +43,8 @@
  * failed launch returns GDN2_ERR_CUDA. gdn2_last_error_string() describes the last
  * failure of the calling thread. Nothing is thrown or aborted across the ABI.
  *
- * Supported: dk, dv in {64, 128}; h_v a multiple of h_qk; every pointer 16-byte aligned.
+ * Supported: dk, dv in {64, 128}; h_v a multiple of h_qk; 1 <= n_seq <= 65535,
+ * h_v <= 65535 and n_seq * h_v <= 2^31 - 1; every pointer 16-byte aligned.
  */
 #ifndef GDN2_H
 #define GDN2_H

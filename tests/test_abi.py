@@ -63,6 +63,8 @@ def test_rejects_before_device_work(lib):
     assert b"dk = 96" in lib.gdn2_last_error_string()
     assert _call_chunk(g, lib, _shape(g, h_qk=3, h_v=4)) == 1
     assert _call_chunk(g, lib, _shape(g, n_seq=0)) == 1
+    assert _call_chunk(g, lib, _shape(g, n_seq=65535, h_qk=65535, h_v=65535)) == 2
+    assert b"pairs above 2^31 - 1" in lib.gdn2_last_error_string()
     assert _call_chunk(g, lib, _shape(g, dtype=7)) == 1
     assert _call_chunk(g, lib, _shape(g, o_dtype=5)) == 1
     assert _call_chunk(g, lib, _shape(g)) == 1  # NULL tensors with T_total > 0
