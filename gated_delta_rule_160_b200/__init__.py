@@ -319,6 +319,37 @@ def gdn2_chunk_bwd(q, k, v, log_alpha, b, w, dO, S0=None, dS_T=None, cu_seqlens=
     return dq, dk, dv, dla, db, dw, dS0
 
 
+class _ChunkFn(torch.autograd.Function):
+    """gdn2_chunk_fwd forward, gdn2_chunk_bwd backward (which recomputes the states from the
+    saved inputs and S0, so nothing but the inputs is kept)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, b, w, S0, cu_seqlens, n_seq):
+        o, S_T = gdn2_chunk_fwd(q, k, v, log_alpha, b, w, S0=S0, cu_seqlens=cu_seqlens, n_seq=n_seq)
+        ctx.save_for_backward(q, k, v, log_alpha, b, w, S0, cu_seqlens)
+        ctx.n_seq = n_seq
+        return o, S_T
+
+    @staticmethod
+    def backward(ctx, dO, dS_T):
+        q, k, v, log_alpha, b, w, S0, cu_seqlens = ctx.saved_tensors
+        dO = torch.zeros(v.shape, dtype=torch.float32, device=v.device) if dO is None else dO.float().contiguous()
+        dS_T = None if dS_T is None else dS_T.float().contiguous()
+        dq, dk, dv, dla, db, dw, dS0 = gdn2_chunk_bwd(
+            q, k, v, log_alpha, b, w, dO, S0=S0, dS_T=dS_T, cu_seqlens=cu_seqlens, n_seq=ctx.n_seq,
+            want_dS0=S0 is not None and ctx.needs_input_grad[6])
+        like = lambda g_, x: g_.to(x.dtype)
+        return (like(dq, q), like(dk, k), like(dv, v), like(dla, log_alpha), like(db, b), like(dw, w), dS0,
+                None, None)
+
+
+def gdn2_chunk(q, k, v, log_alpha, b, w, S0=None, cu_seqlens=None, n_seq=None):
+    """gdn2_chunk_fwd as a differentiable op: returns (o fp32, S_T) and, under autograd,
+    takes the gradients of every input (and of S0) from gdn2_chunk_bwd, cast to each
+    input's dtype. Same shapes and rules as gdn2_chunk_fwd."""
+    return _ChunkFn.apply(q, k, v, log_alpha, b, w, S0, cu_seqlens, n_seq)
+
+
 def gdn2_device_status(stream=None) -> int:
     """Wait for the work queued on ``stream`` (default: the current stream) and return, then
     clear, the device status bits set since the last call (GDN2_DEVICE_* above; 0 = none)."""
