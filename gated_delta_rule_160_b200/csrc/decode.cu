@@ -368,7 +368,6 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
         // the state stays in registers from token to token; no barrier in this loop
         for (int t = 0; t < n_tok; ++t) {
             const size_t row = (size_t)n * n_tok + t;  // token t of sequence n
-            const size_t tv = row * p.h_v + h;
             const float4 *at = reinterpret_cast<const float4*>(sa + t * DK) + rq;
             const float4 *kt = reinterpret_cast<const float4*>(sk + t * DK) + rq;
             const float4 *qt = reinterpret_cast<const float4*>(sq + t * DK) + rq;
@@ -412,7 +411,6 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
             const float4 r = make_float4(r0.x, r0.y, r1.x, r1.y), pq = make_float4(p0.x, p0.y, p1.x, p1.y);
             const float4 x = *reinterpret_cast<const float4*>(sx + t * DV + col);
             const float2 x0 = make_float2(x.x, x.y), x1 = make_float2(x.z, x.w);
-            float* Ss = p.S_steps ? p.S_steps + (row * p.h_v + h) * DK * DV : nullptr;
 #pragma unroll
             for (int j = 0; j < RPT / 4; ++j) {
                 const float4 e4 = et[8 * j], k4 = kt[8 * j];
@@ -424,12 +422,14 @@ __global__ void __launch_bounds__(MultiCfg<DK, DV, T, kPro>::NT, 2)
                     const float2 s0 = ffma2(kv, x0, ffma2(ne, r0, make_float2(si.x, si.y)));
                     const float2 s1 = ffma2(kv, x1, ffma2(ne, r1, make_float2(si.z, si.w)));
                     si = make_float4(s0.x, s0.y, s1.x, s1.y);
-                    if (Ss) __stcs(reinterpret_cast<float4*>(Ss + (size_t)(8 * (4 * j + e) + rq) * DV + col), si);
+                    if (p.S_steps)  // the parameter re-read here keeps no pointer live in the loop
+                        __stcs(reinterpret_cast<float4*>(p.S_steps + (row * p.h_v + h) * DK * DV +
+                                                         (size_t)(8 * (4 * j + e) + rq) * DV + col), si);
                 }
             }
             if (rq == 0) {
                 const float qe = kPro ? dots[t][0] : dq.x, qk = kPro ? dots[t][1] : dq.y;
-                TO* o = static_cast<TO*>(p.o) + tv * DV + col;
+                TO* o = static_cast<TO*>(p.o) + (row * p.h_v + h) * DV + col;
                 o[0] = from_f32<TO>(pq.x - qe * r.x + qk * x.x);
                 o[1] = from_f32<TO>(pq.y - qe * r.y + qk * x.y);
                 o[2] = from_f32<TO>(pq.z - qe * r.z + qk * x.z);
