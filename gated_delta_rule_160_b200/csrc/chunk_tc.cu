@@ -716,16 +716,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 kq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_K + o) : z;
                 bq[pss] = valid ? *reinterpret_cast<const uint2*>(smem + OFF_RAW_B + o) : z;
             }
-            // 1 / |q|, 1 / |k| of this thread's tokens (taken during the previous chunk's solve)
-            float rq[4], rk[4];
-            if (kPro) {
-                const float* rn = reinterpret_cast<const float*>(smem + OFF_RN);
-#pragma unroll
-                for (int pss = 0; pss < 4; ++pss) {
-                    rq[pss] = rn[ti0 + 8 * pss];
-                    rk[pss] = rn[64 + ti0 + 8 * pss];
-                }
-            }
             // the tiles below overwrite Eb, which the previous chunk's U -= R^T Eb MMAs read
             if (ci > 0) fault |= !mbar_wait(mbar(MB_45), par ^ 1u, kWaitNs);
             if (bar_or_1<NS>(fault)) {
@@ -762,10 +752,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_tc_kernel(const __grid_constant__
                 unpack4_bf16(kq[pss], kf);
                 unpack4_bf16(bq[pss], bf);
                 if (kPro) {
+                    // 1 / |q|, 1 / |k| of this token (taken during the previous chunk's solve)
+                    const float* rn = reinterpret_cast<const float*>(smem + OFF_RN);
+                    const float rqv = rn[i], rkv = rn[64 + i];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        qf[e] *= rq[pss];
-                        kf[e] *= rk[pss];
+                        qf[e] *= rqv;
+                        kf[e] *= rkv;
                         bf[e] = sigmoid_tanh_f(bf[e]);  // b only reaches the plain bf16 Eb tile
                     }
                 }
